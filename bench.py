@@ -1,0 +1,504 @@
+"""Benchmark of the HSA denoising step on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+Workload: the full HSA loop of a 30-layer DiT (hidden 1536, 12 heads x 128,
+MLP 8960, bf16 weights N(0, 1/fan_in)) on a 21x30x52 video latent (N = 32760
+tokens x 16 channels), T = 40 flow-matching steps (sigma 1 -> 0, shift 5), K = 3
+groups with budgets {40, 20, 10} holding 40/30/30% of the tokens, re-grouped by
+L1 relative velocity change.  A step is one global iteration i of that loop
+(schedule, embed, 30 sparse layers, head, cached Euler, re-grouping); step k
+runs iteration k mod 40, so 40 steps are one whole loop.  All inputs are seeded
+synthetic data resident in HBM before timing; every step touches > 8 GB
+(weights 2.2 GB + KV caches 6 GB), far more than the 126 MB L2.
+
+One JSON line is printed by rank 0.  ``value`` is ms per denoising step (max
+over ranks; lower is better); extra keys carry the dense all-active step time,
+active-query attention TFLOP/s at 100/50/25% active, cached-Euler GB/s, the
+roofline of the dominant kernel (attention), the end-to-end figure through the
+public call with host buffers, and the CPU oracle timed on a bounded sample.
+With --gpus N > 1 each rank runs an independent replica (the method runs on one
+GPU; there is no data-path collective).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "HSA denoise-step ms & active-query attn TFLOP/s at 25/50/100% active; Euler GB/s"
+WORKLOAD = "dit30_1536"
+
+
+def parse():
+    ap = argparse.ArgumentParser(description="HSA denoising-step benchmark")
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--quick", action="store_true", help="skip the sub-benchmarks (profiling runs)")
+    ap.add_argument("--profile-case", choices=["attention", "gemm", "euler"], default=None,
+                    help="run three launches of one kernel at the workload shape and exit")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------- distributed
+
+def dist_setup(n_gpus):
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+        pg = dist
+    return rank, world, local, pg
+
+
+def max_over_ranks(value: float, pg, device) -> float:
+    if pg is None:
+        return value
+    import torch
+
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(pg):
+    if pg is not None:
+        pg.barrier()
+
+
+# --------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.rows = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 8:
+                self.rows.append(parts)
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if not self.rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[0]) for r in self.rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in self.rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[j] for r in self.rows for j in range(4)
+                          if r[4 + j].lower() == "active"})
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(self.rows)}
+
+
+# --------------------------------------------------------------------------- our arm
+
+def build_loop(spec, seed, torch):
+    from token_sparse_denoising_layer_b200 import synth
+    from token_sparse_denoising_layer_b200.loop import HsaLoop
+
+    sh = spec["shape"]
+    counts = synth.group_counts(sh.N, spec["fractions"])
+    layers = [synth.device_layer_weights(sh.D, sh.F, seed * 1000 + l) for l in range(sh.L)]
+    wf = synth.model_weights(synth.ModelShape(sh.N, sh.C, sh.D, sh.H, 64, 0), seed)
+    w_in = torch.from_numpy(wf["w_in"]).cuda()
+    w_head = torch.from_numpy(wf["w_head"]).cuda()
+    loop = HsaLoop(sh.N, sh.D, sh.H, sh.F, layers, w_in, w_head, spec["T"], spec["budgets"],
+                   counts, shift=spec["shift"])
+    x0 = torch.from_numpy(synth.latent(sh.N, 16, seed)).cuda()
+    g0 = torch.from_numpy(synth.random_split(sh.N, counts, seed)).cuda()
+    return loop, x0, g0, counts, layers
+
+
+def time_steps(loop, steps, torch, regroup=True, per_step_hook=None):
+    """Time `steps` iterations (i = k mod T) with CUDA events on the launch stream."""
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    torch.cuda.synchronize()
+    for k in range(steps):
+        i = k % loop.T
+        ev[k][0].record(stream)
+        if per_step_hook is not None:
+            per_step_hook(k, i)
+        else:
+            loop.step(i, regroup)
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def kernels_per_step(loop, i, regroup=True):
+    """Kernel launches of one hsa_step: schedule, embed, 7 per layer, head, Euler,
+    and 3 for re-grouping when it runs."""
+    n = 4 + 7 * loop.L
+    smin = min(loop.budgets)
+    if regroup and loop.T // smin <= i < loop.T - 1:
+        n += 3 if len(loop.budgets) > 1 else 1
+    return n
+
+
+def attention_sweep(torch, abi, synth):
+    """Single DiT layer, N = 32760, hidden 1536, 12 x 128 heads: attention of
+    |A| = f*N queries against the full cache, f in {1, .5, .25, .1}."""
+    N, D, H = 32760, 1536, 12
+    ctx = abi.hsa_create(N=N, D=D, H=H, F=6144, L=1, T=1, budgets=[1], counts=[N])
+    g = torch.Generator(device="cuda")
+    g.manual_seed(5)
+    kc = torch.randn((N, D), generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn((N, D), generator=g, device="cuda").to(torch.bfloat16)
+    q = torch.randn((N, D), generator=g, device="cuda").to(torch.bfloat16)
+    o = torch.empty((N, D), dtype=torch.bfloat16, device="cuda")
+    out = {}
+    stream = torch.cuda.current_stream()
+    for f in (1.0, 0.5, 0.25, 0.1):
+        a = int(round(f * N))
+        for _ in range(3):
+            abi.hsa_attention(ctx, q, a, kc, vc, o)
+        reps = 10
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for _ in range(reps):
+            abi.hsa_attention(ctx, q, a, kc, vc, o)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        flop = 4.0 * a * N * D
+        out[f"{int(f * 100)}%"] = {"active": a, "ms": round(ms, 4),
+                                   "tflops": round(flop / ms / 1e9, 1)}
+    abi.hsa_sync_check(ctx)
+    ctx.close()
+    return out
+
+
+def euler_bandwidth(torch, abi):
+    """Cached-Euler kernel GB/s at the 21x30x52 and 21x45x80 latents (L2 flushed
+    between samples) and at a 256M-float size (asymptotic)."""
+    res = {}
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    for N in (32760, 75600, 16 * 1024 * 1024):
+        ctx = abi.hsa_create(N=N, D=128, H=1, F=64, L=0, T=40, budgets=[40, 20, 10],
+                             counts=[N - 2 * (N * 3 // 10), N * 3 // 10, N * 3 // 10])
+        x, vh, vp, vf = (torch.randn((N, 16), device="cuda") for _ in range(4))
+        mask = (torch.rand(N, device="cuda") < 0.625).to(torch.uint8)
+        a = int(mask.sum().item())
+        times = []
+        for r in range(13):
+            flush.fill_(float(r))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            abi.hsa_euler_step(ctx, x, vh, vp, vf, mask, 0.5, 0.475)
+            e1.record(stream)
+            torch.cuda.synchronize()
+            if r >= 3:
+                times.append(e0.elapsed_time(e1))
+        ms = float(np.median(times))
+        bytes_ = N * 16 * 4 * 3 + a * 16 * 4 * 3 + N
+        res[str(N)] = {"ms": round(ms, 5), "GBps": round(bytes_ / ms / 1e6, 1), "bytes": bytes_}
+        ctx.close()
+    del flush
+    return res
+
+
+def cpu_baseline(spec, n_rows=64, target_s=12.0):
+    """The oracle on the host cores, on a bounded sample: one layer of the
+    30-layer DiT for `n_rows` active rows against the full N = 32760 cache,
+    repeated until about `target_s` seconds; extrapolated linearly in the
+    active rows to a full step of the loop (cost is O(|A_i|) per layer)."""
+    from oracle import hsa_oracle as O
+    from token_sparse_denoising_layer_b200 import synth
+
+    sh = spec["shape"]
+    r = synth.rng(3)
+    D, F, N = sh.D, sh.F, sh.N
+    w = {"w_qkv": r.standard_normal((3 * D, D), dtype=np.float32) / np.sqrt(D),
+         "w_o": r.standard_normal((D, D), dtype=np.float32) / np.sqrt(D),
+         "w_1": r.standard_normal((F, D), dtype=np.float32) / np.sqrt(D),
+         "w_2": r.standard_normal((D, F), dtype=np.float32) / np.sqrt(F)}
+    x = r.standard_normal((N, D)).astype(np.float64)
+    kc = r.standard_normal((N, D))
+    vc = r.standard_normal((N, D))
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        idx = np.sort(r.permutation(N)[:n_rows]).astype(np.int32)
+        O.layer_forward(w, x, idx, kc, vc, sh.H)
+        reps += 1
+        if time.perf_counter() - t0 >= target_s:
+            break
+    per_row_layer_s = (time.perf_counter() - t0) / (reps * n_rows)
+    counts = synth.group_counts(N, spec["fractions"])
+    mean_active = np.mean([O.n_active(i, spec["T"], spec["budgets"], counts) for i in range(spec["T"])])
+    ms_step = per_row_layer_s * mean_active * sh.L * 1e3
+    try:
+        import torch
+        cores = torch.get_num_threads()
+    except Exception:
+        cores = os.cpu_count()
+    return {"value": round(ms_step, 1), "unit": "ms/step", "cores": cores, "kind": "oracle",
+            "sample": (f"{reps} x oracle layer_forward on {n_rows} active rows vs the full "
+                       f"N={N} cache (D={D}, F={F}); {time.perf_counter() - t0:.1f} s; "
+                       f"extrapolated x{mean_active:.0f} mean active rows x {sh.L} layers")}
+
+
+def run_ours(args, rank, world, local, pg):
+    import torch
+
+    from token_sparse_denoising_layer_b200 import abi, synth
+
+    torch.cuda.set_device(local)
+    spec = synth.WORKLOADS[WORKLOAD]
+    sh = spec["shape"]
+    loop, x0, g0, counts, layers = build_loop(spec, seed=rank, torch=torch)
+
+    # warm-up, then a fresh loop state for the timed region
+    loop.reset(x0, g0)
+    for k in range(args.warmup):
+        loop.step(k % loop.T)
+    abi.hsa_sync_check(loop.ctx)
+    loop.reset(x0, g0)
+    barrier(pg)
+    launches = sum(kernels_per_step(loop, k % loop.T) for k in range(args.steps))
+    with ClockSampler(local) as clk:
+        times = time_steps(loop, args.steps, torch)
+    abi.hsa_sync_check(loop.ctx)
+    ms_total = max_over_ranks(float(np.sum(times)), pg, torch.device("cuda", local))
+    ms_step = ms_total / args.steps
+    barrier(pg)
+
+    # dense all-active loop on the same kernels (every token active every step)
+    dense = None
+    if not args.quick:
+        dl = __import__("token_sparse_denoising_layer_b200.loop", fromlist=["HsaLoop"]).HsaLoop(
+            sh.N, sh.D, sh.H, sh.F, layers, loop.model._keep[0], loop.model._keep[1], spec["T"],
+            [spec["T"]], [sh.N], shift=spec["shift"])
+        dl.reset(x0, torch.zeros_like(g0))
+        for k in range(2):
+            dl.step(k)
+        dl.reset(x0, torch.zeros_like(g0))
+        dt = time_steps(dl, min(args.steps, 8), torch)
+        dense = float(np.mean(dt))
+        dl.close()
+        del dl
+
+    # end to end through the public call with host buffers: H2D of the latent,
+    # the step, D2H of the latent, every step
+    # (two pinned host buffers ping-pong, so the latent really travels through host memory)
+    x_host = [torch.empty((sh.N, 16), dtype=torch.float32).pin_memory() for _ in range(2)]
+    x_host[0].copy_(x0.cpu())
+    loop.reset(x0, g0)
+
+    def e2e_hook(k, i):
+        loop.x.copy_(x_host[k % 2], non_blocking=True)
+        loop.step(i)
+        x_host[(k + 1) % 2].copy_(loop.x, non_blocking=True)
+
+    e2e_times = time_steps(loop, args.steps, torch, per_step_hook=e2e_hook)
+    e2e_ms = max_over_ranks(float(np.sum(e2e_times)), pg, torch.device("cuda", local)) / args.steps
+
+    sub = {}
+    if not args.quick and rank == 0:
+        sub["attention"] = attention_sweep(torch, abi, synth)
+        sub["euler"] = euler_bandwidth(torch, abi)
+
+    result = None
+    if rank == 0:
+        peaks = {}
+        pp = os.path.join(ROOT, "MEASURED_PEAKS.json")
+        if os.path.exists(pp):
+            with open(pp) as f:
+                peaks = json.load(f)
+        peak_tf = peaks.get("bf16_tflops_sustained", 1400.0)
+        roof = None
+        if "attention" in sub:
+            a100 = sub["attention"]["100%"]
+            roof = {"bound": "tensor", "kernel": "k_attn<128> (active-query attention)",
+                    "achieved": a100["tflops"], "peak": peak_tf, "unit": "TFLOP/s",
+                    "frac": round(a100["tflops"] / peak_tf, 3),
+                    "peak_source": "MEASURED_PEAKS.json bf16_tflops_sustained (of measured)"
+                    if "bf16_tflops_sustained" in peaks else "fallback 1400 TFLOP/s",
+                    "traffic": None,
+                    "per_launch": "4*|A|*N*D FLOP, |A| = N = 32760, D = 1536"}
+        result = {
+            "metric": METRIC, "value": round(ms_step, 3), "unit": "ms/step", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; random N(0,1/fan_in) weights, x ~ N(0,1))",
+            "config": {"workload": "HSA loop, 30-layer DiT: N=32760 (21x30x52), C=16, D=1536, "
+                                   "H=12x128, F=8960, T=40, shift 5, budgets {40,20,10} at "
+                                   "40/30/30%, regroup by L1 relative velocity change",
+                       "global_batch": 1, "seq_len": sh.N, "parallelism": f"replicas x{world}",
+                       "l2": "inputs larger than L2 (>8 GB touched per step)",
+                       "step": "one global iteration i = k mod 40; 40 steps = one loop"},
+            "dense_ms_per_step": round(dense, 3) if dense else None,
+            "hsa_vs_dense": round(ms_step / dense, 3) if dense else None,
+            "mean_active_fraction": 0.625,
+            "gpu_launches": launches,
+            "e2e": {"value": round(e2e_ms, 3), "unit": "ms/step",
+                    "h2d_bytes_per_step": sh.N * 16 * 4, "d2h_bytes_per_step": sh.N * 16 * 4},
+            "clocks": clk.summary(),
+            "roofline": roof,
+            "sub": sub,
+        }
+        if not args.no_cpu_baseline and world == 1:
+            result["cpu_baseline"] = cpu_baseline(spec)
+    loop.close()
+    return result
+
+
+# --------------------------------------------------------------------------- reference arm
+
+def run_reference(args, rank, world):
+    """The CPU oracle as the reference arm: each step a bounded sample of the
+    same workload (8 active rows of one layer, extrapolated to the step)."""
+    if rank != 0:
+        return None
+    from oracle import hsa_oracle as O
+    from token_sparse_denoising_layer_b200 import synth
+
+    spec = synth.WORKLOADS[WORKLOAD]
+    sh = spec["shape"]
+    r = synth.rng(4)
+    D, F, N = sh.D, sh.F, sh.N
+    w = {"w_qkv": r.standard_normal((3 * D, D), dtype=np.float32) / np.sqrt(D),
+         "w_o": r.standard_normal((D, D), dtype=np.float32) / np.sqrt(D),
+         "w_1": r.standard_normal((F, D), dtype=np.float32) / np.sqrt(D),
+         "w_2": r.standard_normal((D, F), dtype=np.float32) / np.sqrt(F)}
+    x = r.standard_normal((N, D))
+    kc, vc = r.standard_normal((N, D)), r.standard_normal((N, D))
+    counts = synth.group_counts(N, spec["fractions"])
+    rows = 8
+    per_step = []
+    for k in range(args.warmup + args.steps):
+        i = k % spec["T"]
+        a = O.n_active(i, spec["T"], spec["budgets"], counts)
+        idx = np.sort(r.permutation(N)[:rows]).astype(np.int32)
+        t0 = time.perf_counter()
+        O.layer_forward(w, x, idx, kc, vc, sh.H)
+        t = time.perf_counter() - t0
+        if k >= args.warmup:
+            per_step.append(t / rows * a * sh.L * 1e3)
+    ms = float(np.mean(per_step))
+    try:
+        import torch
+        cores = torch.get_num_threads()
+    except Exception:
+        cores = os.cpu_count()
+    return {"impl": "reference", "metric": METRIC, "value": round(ms, 1), "unit": "ms/step",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(ms, 1), "higher_is_better": False, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "HSA loop, 30-layer DiT: N=32760, D=1536, H=12x128, F=8960, "
+                                   "T=40, budgets {40,20,10} at 40/30/30%"},
+            "cpu_baseline": {"value": round(ms, 1), "unit": "ms/step", "cores": cores,
+                             "kind": "oracle",
+                             "sample": f"per step: oracle layer_forward on {rows} active rows of "
+                                       f"one layer vs the full cache, extrapolated by |A_i| x {sh.L} layers"},
+            "e2e": {"value": round(ms, 1), "unit": "ms/step", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def profile_case(name):
+    """A few launches of one kernel at the workload's shapes, for ncu captures."""
+    import torch
+
+    from token_sparse_denoising_layer_b200 import abi
+
+    N, D, H, F = 32760, 1536, 12, 8960
+    ctx = abi.hsa_create(N=N, D=D, H=H, F=F, L=1, T=40, budgets=[40, 20, 10],
+                         counts=[13104, 9828, 9828])
+    g = torch.Generator(device="cuda")
+    g.manual_seed(1)
+    rnd = lambda *s: torch.randn(s, generator=g, device="cuda")
+    if name == "attention":
+        kc, vc, q = (rnd(N, D).to(torch.bfloat16) for _ in range(3))
+        o = torch.empty_like(q)
+        for _ in range(3):
+            abi.hsa_attention(ctx, q, N, kc, vc, o)
+    elif name == "gemm":
+        u = rnd(N, D).to(torch.bfloat16)
+        w1 = (rnd(F, D) / D ** 0.5).to(torch.bfloat16)
+        out = torch.empty((N, F), dtype=torch.bfloat16, device="cuda")
+        for _ in range(3):
+            abi.hsa_linear(ctx, u, N, D, w1, F, out)
+    elif name == "euler":
+        x, vh, vp, vf = (rnd(N, 16) for _ in range(4))
+        m = (torch.rand(N, device="cuda") < 0.6).to(torch.uint8)
+        for _ in range(3):
+            abi.hsa_euler_step(ctx, x, vh, vp, vf, m, 0.5, 0.45)
+    abi.hsa_sync_check(ctx)
+    ctx.close()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.profile_case:
+        return profile_case(args.profile_case)
+    if args.impl == "reference":
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        res = run_reference(args, rank, world)
+        if rank == 0 and res is not None:
+            print(json.dumps(res), flush=True)
+        return 0
+    rank, world, local, pg = dist_setup(args.gpus)
+    res = run_ours(args, rank, world, local, pg)
+    if rank == 0 and res is not None:
+        print(json.dumps(res), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -31,7 +31,7 @@ from scipy.special import erf as _erf
 __all__ = [
     "check_budgets", "strides", "active_mask", "active_index", "n_active",
     "l1_relative_change", "l1_relative_change_f64", "rank_keys_order",
-    "assign_groups", "sigma_schedule", "layer_norm", "gelu", "bf16",
+    "assign_groups", "sigma_schedule", "linear", "layer_norm", "gelu", "bf16",
     "attention", "layer_forward", "embed", "head", "euler_step",
     "euler_step_f32", "regroup_from", "run_loop", "dense_loop",
 ]
@@ -181,6 +181,11 @@ def bf16(a: np.ndarray) -> np.ndarray:
     u = f.view(np.uint32).astype(np.uint64)
     u = (u + 0x7FFF + ((u >> 16) & 1)) >> 16 << 16
     return u.astype(np.uint32).view(np.float32).astype(np.float64).reshape(f.shape)
+
+
+def linear(a: np.ndarray, w: np.ndarray) -> np.ndarray:
+    """Active-row linear map a w^T with w in Linear layout [out, in] ([TS] 2.2)."""
+    return np.asarray(a, dtype=np.float64) @ np.asarray(w, dtype=np.float64).T
 
 
 def layer_norm(x: np.ndarray, eps: float = LN_EPS) -> np.ndarray:

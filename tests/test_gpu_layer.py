@@ -1,0 +1,201 @@
+"""GPU parity of the tensor-core path against the oracle: active-row GEMMs,
+LayerNorm gather, KV-cache write, active-query attention, and the whole
+sparse transformer block.  bf16 storage with fp32 accumulation; outputs must
+be within 1e-2 normwise (max|gpu - ref| / max|ref|) of the float64 oracle.
+Sizes span several 128-row tiles with ragged tails in both the query and the
+key dimension.
+"""
+
+import numpy as np
+import pytest
+
+from gpu_util import BF16_TOL, bf, dev, host, need_gpu, normwise, torch
+from oracle import hsa_oracle as O
+from token_sparse_denoising_layer_b200 import abi, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def _ctx(N, D, H, F):
+    return abi.hsa_create(N=N, D=D, H=H, F=F, L=1, T=1, budgets=[1], counts=[N])
+
+
+@pytest.mark.parametrize("M,K,Ncols", [(1, 64, 32), (128, 128, 256), (333, 256, 384),
+                                       (700, 1536, 4608), (129, 512, 1536), (5, 6144, 128)])
+def test_linear(M, K, Ncols):
+    need_gpu()
+    ctx = _ctx(max(M, 1), 128, 1, 64)
+    r = synth.rng(M + K)
+    a = synth.bf16_round(r.standard_normal((M, K), dtype=np.float32))
+    w = synth.bf16_round(r.standard_normal((Ncols, K), dtype=np.float32) / np.sqrt(K))
+    out = torch.empty((M, Ncols), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_linear(ctx, bf(a), M, K, bf(w), Ncols, out)
+    abi.hsa_sync_check(ctx)
+    assert normwise(host(out), O.linear(a, w)) <= BF16_TOL
+
+
+def test_linear_rejects_bad_shape():
+    need_gpu()
+    ctx = _ctx(16, 128, 1, 64)
+    a = torch.zeros((16, 100), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(abi.HsaError):
+        abi.hsa_linear(ctx, a, 16, 100, a, 32, a)
+
+
+@pytest.mark.parametrize("N,D,a", [(700, 256, 333), (1000, 1536, 129), (64, 5120, 64)])
+def test_ln_gather(N, D, a):
+    need_gpu()
+    ctx = _ctx(N, D, D // 128, 64)
+    x = synth.hidden_rows(N, D, 1) * np.float32(3) + np.float32(0.5)
+    idx = synth.random_active_set(N, a, 1)
+    u = torch.empty((a, D), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_ln_gather(ctx, dev(x), dev(idx), a, u)
+    abi.hsa_sync_check(ctx)
+    assert normwise(host(u), O.layer_norm(x[idx])) <= 4e-3
+
+
+@pytest.mark.parametrize("N,D,H,n,q_scale", [
+    (700, 256, 2, 333, 4.0),      # 6 key tiles (tail 60), 3 query tiles (tail 77)
+    (1000, 128, 2, 1000, 1.0),    # head_dim 64
+    (130, 128, 1, 1, 8.0),        # one query, key tail of 2
+    (4096, 1536, 12, 200, 3.0),
+])
+def test_attention(N, D, H, n, q_scale):
+    need_gpu()
+    ctx = _ctx(N, D, H, 64)
+    q, k, v = synth.attention_inputs(n, N, D, 2, q_scale=q_scale)
+    o = torch.empty((n, D), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_attention(ctx, bf(q), n, bf(k), bf(v), o)
+    abi.hsa_sync_check(ctx)
+    ref = O.attention(q, k, v, H)
+    assert normwise(host(o), ref) <= BF16_TOL
+
+
+def test_attention_identical_keys_mean_of_values():
+    need_gpu()
+    N, D, H, n = 300, 128, 1, 130
+    ctx = _ctx(N, D, H, 64)
+    q, _, v = synth.attention_inputs(n, N, D, 3, q_scale=5.0)
+    k = np.tile(q[:1], (N, 1))
+    o = torch.empty((n, D), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_attention(ctx, bf(q), n, bf(k), bf(v), o)
+    assert normwise(host(o), np.tile(v.astype(np.float64).mean(axis=0), (n, 1))) <= BF16_TOL
+
+
+def test_kv_scatter_and_qkv_project():
+    need_gpu()
+    N, D, H, a = 700, 256, 2, 333
+    ctx = _ctx(N, D, H, 64)
+    w = synth.layer_weights(D, 64, 4)
+    x = synth.hidden_rows(N, D, 4)
+    ks, vs = synth.stale_kv(N, D, 4)
+    idx = synth.random_active_set(N, a, 4)
+    u = torch.empty((a, D), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_ln_gather(ctx, dev(x), dev(idx), a, u)
+    q = torch.empty((a, D), dtype=torch.bfloat16, device="cuda")
+    kc, vc = bf(ks), bf(vs)
+    abi.hsa_qkv_project(ctx, bf(w["w_qkv"]), u, dev(idx), a, q, kc, vc)
+    abi.hsa_sync_check(ctx)
+    qkv = O.linear(O.layer_norm(x[idx]), w["w_qkv"])
+    assert normwise(host(q), qkv[:, :D]) <= BF16_TOL
+    kh, vh = host(kc), host(vc)
+    assert normwise(kh[idx], qkv[:, D:2 * D]) <= BF16_TOL
+    assert normwise(vh[idx], qkv[:, 2 * D:]) <= BF16_TOL
+    rest = np.setdiff1d(np.arange(N), idx)
+    assert (kh[rest] == ks[rest]).all() and (vh[rest] == vs[rest]).all()
+    # standalone scatter: bit-exact copy
+    kr = synth.bf16_round(synth.rng(9).standard_normal((a, D), dtype=np.float32))
+    kc2, vc2 = bf(ks), bf(vs)
+    abi.hsa_kv_scatter(ctx, bf(kr), bf(-kr), dev(idx), a, kc2, vc2)
+    want_k = ks.copy()
+    want_k[idx] = kr
+    assert (host(kc2) == want_k).all()
+    assert (host(vc2)[idx] == -kr).all()
+
+
+@pytest.mark.parametrize("N,D,H,F,a", [(700, 256, 2, 512, 333), (256, 128, 2, 512, 128),
+                                       (1500, 1536, 12, 6144, 260)])
+def test_layer_forward(N, D, H, F, a):
+    need_gpu()
+    ctx = _ctx(N, D, H, F)
+    w = synth.layer_weights(D, F, 6)
+    x = synth.hidden_rows(N, D, 6)
+    ks, vs = synth.stale_kv(N, D, 6)
+    idx = synth.random_active_set(N, a, 6)
+    xd, kc, vc = dev(x), bf(ks), bf(vs)
+    lw = abi.layer_weights(*(bf(w[k]) for k in ("w_qkv", "w_o", "w_1", "w_2")))
+    abi.hsa_layer_forward(ctx, lw, xd, dev(idx), a, kc, vc)
+    abi.hsa_sync_check(ctx)
+    xr = x.astype(np.float64).copy()
+    kr, vr = ks.astype(np.float64).copy(), vs.astype(np.float64).copy()
+    tr = {}
+    O.layer_forward(w, xr, idx, kr, vr, H, trace=tr)
+    xg = host(xd)
+    rest = np.setdiff1d(np.arange(N), idx)
+    assert (xg[rest] == x[rest]).all()
+    assert normwise(xg[idx] - x[idx], xr[idx] - x[idx]) <= BF16_TOL
+    assert normwise(host(kc)[idx], kr[idx]) <= BF16_TOL
+    assert normwise(host(vc)[idx], vr[idx]) <= BF16_TOL
+
+
+def test_layer_forward_empty_active_set_is_noop():
+    need_gpu()
+    N, D, H, F = 256, 128, 2, 512
+    ctx = _ctx(N, D, H, F)
+    x = synth.hidden_rows(N, D, 7)
+    xd = dev(x)
+    w = synth.layer_weights(D, F, 7)
+    lw = abi.layer_weights(*(bf(w[k]) for k in ("w_qkv", "w_o", "w_1", "w_2")))
+    kc = torch.zeros((N, D), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_layer_forward(ctx, lw, xd, dev(np.zeros(1, np.int32)), 0, kc, kc.clone())
+    assert (host(xd) == x).all()
+
+
+def test_bad_index_is_reported_not_faulted():
+    need_gpu()
+    N, D = 256, 128
+    ctx = _ctx(N, D, 2, 512)
+    x = dev(synth.hidden_rows(N, D, 8))
+    idx = np.array([1, 2, 300], dtype=np.int32)   # 300 >= N
+    u = torch.empty((3, D), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_ln_gather(ctx, x, dev(idx), 3, u)
+    with pytest.raises(abi.HsaError) as e:
+        abi.hsa_sync_check(ctx)
+    assert e.value.status == 7
+
+
+@pytest.mark.parametrize("N,D,H,F,a", [(700, 256, 2, 512, 333), (1500, 1536, 12, 6144, 260)])
+def test_layer_stages(N, D, H, F, a):
+    """Each stage of the block through its own entry point, against the oracle's trace."""
+    need_gpu()
+    ctx = _ctx(N, D, H, F)
+    w = synth.layer_weights(D, F, 6)
+    x = synth.hidden_rows(N, D, 6)
+    ks, vs = synth.stale_kv(N, D, 6)
+    idx = synth.random_active_set(N, a, 6)
+    xr = x.astype(np.float64).copy()
+    kr, vr = ks.astype(np.float64).copy(), vs.astype(np.float64).copy()
+    tr = {}
+    O.layer_forward(w, xr, idx, kr, vr, H, trace=tr)
+    xd, kc, vc, idd = dev(x), bf(ks), bf(vs), dev(idx)
+    u = torch.empty((a, D), dtype=torch.bfloat16, device="cuda")
+    q = torch.empty_like(u)
+    o = torch.empty_like(u)
+    errs = {}
+    abi.hsa_ln_gather(ctx, xd, idd, a, u)
+    errs["u"] = normwise(host(u), tr["u"])
+    abi.hsa_qkv_project(ctx, bf(w["w_qkv"]), u, idd, a, q, kc, vc)
+    errs["q"] = normwise(host(q), tr["q"])
+    errs["k"] = normwise(host(kc)[idx], tr["k"])
+    abi.hsa_attention(ctx, q, a, kc, vc, o)
+    errs["o"] = normwise(host(o), tr["o"])
+    abi.hsa_out_proj_residual(ctx, bf(w["w_o"]), o, idd, a, xd)
+    x1_ref = x[idx].astype(np.float64) + O.linear(tr["o"], w["w_o"])
+    errs["attn_delta"] = normwise(host(xd)[idx] - x[idx], x1_ref - x[idx])
+    x1 = host(xd)[idx].copy()
+    abi.hsa_mlp_residual(ctx, bf(w["w_1"]), bf(w["w_2"]), xd, idd, a)
+    mlp_ref = O.linear(O.gelu(O.linear(O.layer_norm(x1), w["w_1"])), w["w_2"])
+    errs["mlp_delta"] = normwise(host(xd)[idx] - x1, mlp_ref)
+    print(errs)
+    abi.hsa_sync_check(ctx)
+    assert all(e <= BF16_TOL for e in errs.values()), errs

@@ -1,0 +1,83 @@
+"""The whole HSA loop on the GPU (hsa_step) against the oracle's loop, on the
+tiny DiT workload (4x8x8 latent, N=256, 2 layers, T=8, budgets {8, 4}).
+
+The GPU runs the layers in bf16 and the oracle in float64, so the latents
+drift apart by rounding; the drift after T steps is stated and bounded here.
+With re-grouping on, a rounding difference can move a token whose score sits
+on a group boundary, so that run is checked for valid groups and a looser drift.
+"""
+
+import numpy as np
+import pytest
+
+from gpu_util import bf, dev, host, need_gpu, torch
+from oracle import hsa_oracle as O
+from token_sparse_denoising_layer_b200 import abi, synth
+from token_sparse_denoising_layer_b200.loop import HsaLoop, sigma_schedule
+
+pytestmark = pytest.mark.gpu
+
+
+def _setup(budgets=(8, 4), fractions=(0.5, 0.5)):
+    spec = synth.WORKLOADS["tiny_dit"]
+    sh = spec["shape"]
+    T = spec["T"]
+    counts = synth.group_counts(sh.N, fractions)
+    w = synth.model_weights(sh, spec["seed"])
+    layers = [tuple(bf(lw[k]) for k in ("w_qkv", "w_o", "w_1", "w_2")) for lw in w["layers"]]
+    loop = HsaLoop(sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]), T,
+                   list(budgets), counts, shift=spec["shift"])
+    x0 = synth.latent(sh.N, 16, spec["seed"])
+    g0 = synth.random_split(sh.N, counts, spec["seed"])
+    return sh, T, counts, w, loop, x0, g0
+
+
+def _drift(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+def test_sigma_tables_agree():
+    for T, s in ((8, 1.0), (40, 5.0)):
+        assert (sigma_schedule(T, s) == O.sigma_schedule(T, s)).all()
+
+
+@pytest.mark.parametrize("regroup", [False, True])
+def test_tiny_dit_loop_drift(regroup):
+    need_gpu()
+    sh, T, counts, w, loop, x0, g0 = _setup()
+    loop.reset(x0, g0)
+    loop.run(regroup=regroup)
+    abi.hsa_sync_check(loop.ctx)
+    xg = host(loop.x)
+    g_end = host(loop.g)
+    assert [int((g_end == k).sum()) for k in range(2)] == counts
+    xr = O.run_loop(w, x0, g0, T, [8, 4], counts, O.sigma_schedule(T, 1.0), sh.H, regroup=regroup)
+    d = _drift(xg, xr)
+    print(f"tiny DiT x_T drift vs float64 oracle (regroup={regroup}): {d:.3e}")
+    assert d <= (2e-2 if not regroup else 5e-2)
+
+
+def test_all_active_loop_matches_dense_oracle():
+    """Every s_k = T: the GPU loop is uniform flow matching; compared with the
+    oracle's dense loop (no KV cache, no velocity cache)."""
+    need_gpu()
+    sh, T, counts, w, loop, x0, g0 = _setup(budgets=(8,), fractions=(1.0,))
+    loop.reset(x0, np.zeros(sh.N, dtype=np.uint8))
+    loop.run()
+    xr = O.dense_loop(w, x0, T, O.sigma_schedule(T, 1.0), sh.H)
+    d = _drift(host(loop.x), xr)
+    print(f"all-active loop drift vs dense oracle: {d:.3e}")
+    assert d <= 2e-2
+
+
+def test_loop_is_deterministic():
+    need_gpu()
+    sh, T, counts, w, loop, x0, g0 = _setup()
+    loop.reset(x0, g0)
+    loop.run()
+    a = host(loop.x).copy()
+    loop.reset(x0, g0)
+    for kc in loop.k_cache + loop.v_cache:
+        kc.zero_()
+    loop.run()
+    assert (host(loop.x) == a).all()

@@ -1,0 +1,273 @@
+"""Thin ctypes binding of libhsa.so: the same names as the C ABI in include/hsa.h.
+
+Only argument marshalling happens here.  Tensors are passed by device
+address (``tensor.data_ptr()``); every step of the HSA path runs in the
+library's CUDA kernels.  There is no fallback: if libhsa.so is missing, or a
+call fails, an exception is raised.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Sequence
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libhsa.so")
+
+# Every symbol the header declares, in header order.
+SYMBOLS = [
+    "hsa_create", "hsa_destroy", "hsa_last_error", "hsa_set_stream", "hsa_sync_check",
+    "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
+    "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_linear", "hsa_kv_scatter",
+    "hsa_attention", "hsa_out_proj_residual", "hsa_mlp_residual", "hsa_layer_forward",
+    "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_step",
+]
+
+STATUS = {0: "HSA_OK", 1: "HSA_ERR_INVALID_ARG", 2: "HSA_ERR_BUDGET", 3: "HSA_ERR_SHAPE",
+          4: "HSA_ERR_CUDA", 5: "HSA_ERR_OOM", 6: "HSA_ERR_TIMEOUT", 7: "HSA_ERR_DEVICE_CHECK"}
+
+
+class HsaError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"{STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+class hsa_model_cfg(ctypes.Structure):
+    _fields_ = [("N", ctypes.c_int), ("C", ctypes.c_int), ("D", ctypes.c_int),
+                ("H", ctypes.c_int), ("F", ctypes.c_int), ("L", ctypes.c_int)]
+
+
+class hsa_layer_weights(ctypes.Structure):
+    _fields_ = [("w_qkv", ctypes.c_void_p), ("w_o", ctypes.c_void_p),
+                ("w_1", ctypes.c_void_p), ("w_2", ctypes.c_void_p)]
+
+
+class hsa_model_weights(ctypes.Structure):
+    _fields_ = [("w_in", ctypes.c_void_p), ("w_head", ctypes.c_void_p),
+                ("layers", ctypes.POINTER(hsa_layer_weights))]
+
+
+class hsa_state(ctypes.Structure):
+    _fields_ = [("x", ctypes.c_void_p), ("v_hat", ctypes.c_void_p),
+                ("v_hat_prev", ctypes.c_void_p), ("v_fresh", ctypes.c_void_p),
+                ("score", ctypes.c_void_p), ("g", ctypes.c_void_p), ("mask", ctypes.c_void_p),
+                ("active_idx", ctypes.c_void_p), ("h", ctypes.c_void_p),
+                ("k_cache", ctypes.POINTER(ctypes.c_void_p)),
+                ("v_cache", ctypes.POINTER(ctypes.c_void_p))]
+
+
+_lib = None
+
+
+def load() -> ctypes.CDLL:
+    """Load libhsa.so (built in-tree by ``token_sparse_denoising_layer_b200.build``)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                           "`python -m token_sparse_denoising_layer_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, I, F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    sig = {
+        "hsa_create": (I, [ctypes.POINTER(hsa_model_cfg), I, ctypes.POINTER(I), ctypes.POINTER(I),
+                           I, I, P, ctypes.POINTER(P)]),
+        "hsa_destroy": (None, [P]),
+        "hsa_last_error": (ctypes.c_char_p, [P]),
+        "hsa_set_stream": (I, [P, P]),
+        "hsa_sync_check": (I, [P]),
+        "hsa_n_active": (I, [P, I]),
+        "hsa_schedule": (I, [P, I, P, P, P, P, ctypes.POINTER(I)]),
+        "hsa_score": (I, [P, P, P, P]),
+        "hsa_select_from_score": (I, [P, P, P]),
+        "hsa_select_groups": (I, [P, P, P, P, P]),
+        "hsa_ln_gather": (I, [P, P, P, I, P]),
+        "hsa_qkv_project": (I, [P, P, P, P, I, P, P, P]),
+        "hsa_linear": (I, [P, P, I, I, P, I, P]),
+        "hsa_kv_scatter": (I, [P, P, P, P, I, P, P]),
+        "hsa_attention": (I, [P, P, I, P, P, P]),
+        "hsa_out_proj_residual": (I, [P, P, P, P, I, P]),
+        "hsa_mlp_residual": (I, [P, P, P, P, P, I]),
+        "hsa_layer_forward": (I, [P, ctypes.POINTER(hsa_layer_weights), P, P, I, P, P]),
+        "hsa_embed": (I, [P, P, P, P, I, P]),
+        "hsa_head": (I, [P, P, P, P, I, P]),
+        "hsa_euler_step": (I, [P, P, P, P, P, P, F, F]),
+        "hsa_step": (I, [P, ctypes.POINTER(hsa_model_weights), ctypes.POINTER(hsa_state), I, F, F, I]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _p(t) -> Optional[int]:
+    """Device address of a tensor (None passes NULL)."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libhsa takes CUDA tensors")
+    if not t.is_contiguous():
+        raise ValueError("libhsa takes contiguous tensors")
+    return t.data_ptr()
+
+
+def _check(ctx, status: int) -> None:
+    if status != 0:
+        msg = load().hsa_last_error(ctx)
+        raise HsaError(status, msg.decode() if msg else "")
+
+
+class Context:
+    """Owns an ``hsa_ctx*``; the handle is ``.ptr``.  Destroyed with ``close()`` or on GC."""
+
+    def __init__(self, ptr: int, cfg: hsa_model_cfg):
+        self.ptr = ptr
+        self.cfg = cfg
+
+    def close(self) -> None:
+        if self.ptr:
+            load().hsa_destroy(self.ptr)
+            self.ptr = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def _stream_ptr(stream) -> Optional[int]:
+    if stream is None:
+        import torch
+        stream = torch.cuda.current_stream()
+    return getattr(stream, "cuda_stream", stream) or None
+
+
+def hsa_create(N: int, D: int, H: int, F: int, L: int, T: int, budgets: Sequence[int],
+               counts: Sequence[int], m: int = 0, C: int = 16, stream=None) -> Context:
+    lib = load()
+    K = len(budgets)
+    cfg = hsa_model_cfg(N, C, D, H, F, L)
+    b = (ctypes.c_int * K)(*budgets)
+    c = (ctypes.c_int * K)(*counts)
+    out = ctypes.c_void_p()
+    st = lib.hsa_create(ctypes.byref(cfg), T, b, c, K, m, _stream_ptr(stream), ctypes.byref(out))
+    _check(None, st)
+    return Context(out.value, cfg)
+
+
+def hsa_destroy(ctx: Context) -> None:
+    ctx.close()
+
+
+def hsa_set_stream(ctx: Context, stream) -> None:
+    _check(ctx.ptr, load().hsa_set_stream(ctx.ptr, _stream_ptr(stream)))
+
+
+def hsa_sync_check(ctx: Context) -> None:
+    _check(ctx.ptr, load().hsa_sync_check(ctx.ptr))
+
+
+def hsa_n_active(ctx: Context, i: int) -> int:
+    return load().hsa_n_active(ctx.ptr, i)
+
+
+def hsa_schedule(ctx: Context, i: int, g, mask, active_idx, n_active_dev=None) -> int:
+    n = ctypes.c_int(0)
+    _check(ctx.ptr, load().hsa_schedule(ctx.ptr, i, _p(g), _p(mask), _p(active_idx),
+                                        _p(n_active_dev), ctypes.byref(n)))
+    return n.value
+
+
+def hsa_score(ctx: Context, v_prev, v_cur, score) -> None:
+    _check(ctx.ptr, load().hsa_score(ctx.ptr, _p(v_prev), _p(v_cur), _p(score)))
+
+
+def hsa_select_from_score(ctx: Context, score, g) -> None:
+    _check(ctx.ptr, load().hsa_select_from_score(ctx.ptr, _p(score), _p(g)))
+
+
+def hsa_select_groups(ctx: Context, v_prev, v_cur, score, g) -> None:
+    _check(ctx.ptr, load().hsa_select_groups(ctx.ptr, _p(v_prev), _p(v_cur), _p(score), _p(g)))
+
+
+def hsa_ln_gather(ctx: Context, x, idx, n: int, u) -> None:
+    _check(ctx.ptr, load().hsa_ln_gather(ctx.ptr, _p(x), _p(idx), n, _p(u)))
+
+
+def hsa_qkv_project(ctx: Context, w_qkv, u, idx, n: int, q, k_cache, v_cache) -> None:
+    _check(ctx.ptr, load().hsa_qkv_project(ctx.ptr, _p(w_qkv), _p(u), _p(idx), n, _p(q),
+                                           _p(k_cache), _p(v_cache)))
+
+
+def hsa_linear(ctx: Context, a, M: int, Kd: int, w, Ncols: int, out) -> None:
+    _check(ctx.ptr, load().hsa_linear(ctx.ptr, _p(a), M, Kd, _p(w), Ncols, _p(out)))
+
+
+def hsa_kv_scatter(ctx: Context, k_rows, v_rows, idx, n: int, k_cache, v_cache) -> None:
+    _check(ctx.ptr, load().hsa_kv_scatter(ctx.ptr, _p(k_rows), _p(v_rows), _p(idx), n,
+                                          _p(k_cache), _p(v_cache)))
+
+
+def hsa_attention(ctx: Context, q, n: int, k_cache, v_cache, o) -> None:
+    _check(ctx.ptr, load().hsa_attention(ctx.ptr, _p(q), n, _p(k_cache), _p(v_cache), _p(o)))
+
+
+def hsa_out_proj_residual(ctx: Context, w_o, o, idx, n: int, x) -> None:
+    _check(ctx.ptr, load().hsa_out_proj_residual(ctx.ptr, _p(w_o), _p(o), _p(idx), n, _p(x)))
+
+
+def hsa_mlp_residual(ctx: Context, w_1, w_2, x, idx, n: int) -> None:
+    _check(ctx.ptr, load().hsa_mlp_residual(ctx.ptr, _p(w_1), _p(w_2), _p(x), _p(idx), n))
+
+
+def layer_weights(w_qkv, w_o, w_1, w_2) -> hsa_layer_weights:
+    """The struct holds raw device addresses, so it also keeps the tensors alive."""
+    s = hsa_layer_weights(_p(w_qkv), _p(w_o), _p(w_1), _p(w_2))
+    s._keep = (w_qkv, w_o, w_1, w_2)
+    return s
+
+
+def hsa_layer_forward(ctx: Context, w: hsa_layer_weights, x, idx, n: int, k_cache, v_cache) -> None:
+    _check(ctx.ptr, load().hsa_layer_forward(ctx.ptr, ctypes.byref(w), _p(x), _p(idx), n,
+                                             _p(k_cache), _p(v_cache)))
+
+
+def hsa_embed(ctx: Context, w_in, x_lat, idx, n: int, h) -> None:
+    _check(ctx.ptr, load().hsa_embed(ctx.ptr, _p(w_in), _p(x_lat), _p(idx), n, _p(h)))
+
+
+def hsa_head(ctx: Context, w_head, h, idx, n: int, v_fresh) -> None:
+    _check(ctx.ptr, load().hsa_head(ctx.ptr, _p(w_head), _p(h), _p(idx), n, _p(v_fresh)))
+
+
+def hsa_euler_step(ctx: Context, x, v_hat, v_hat_prev, v_fresh, mask, sigma_i: float,
+                   sigma_next: float) -> None:
+    _check(ctx.ptr, load().hsa_euler_step(ctx.ptr, _p(x), _p(v_hat), _p(v_hat_prev), _p(v_fresh),
+                                          _p(mask), float(sigma_i), float(sigma_next)))
+
+
+class ModelBinding:
+    """Keeps the ctypes structs of hsa_step (weights and state) alive."""
+
+    def __init__(self, w_in, w_head, layers, x, v_hat, v_hat_prev, v_fresh, score, g, mask,
+                 active_idx, h, k_caches, v_caches):
+        L = len(layers)
+        self._layers = (hsa_layer_weights * max(L, 1))(*[layer_weights(*lw) for lw in layers])
+        self.weights = hsa_model_weights(_p(w_in), _p(w_head), self._layers)
+        self._kc = (ctypes.c_void_p * max(L, 1))(*[_p(t) for t in k_caches])
+        self._vc = (ctypes.c_void_p * max(L, 1))(*[_p(t) for t in v_caches])
+        self.state = hsa_state(_p(x), _p(v_hat), _p(v_hat_prev), _p(v_fresh), _p(score), _p(g),
+                               _p(mask), _p(active_idx), _p(h), self._kc, self._vc)
+        self._keep = (w_in, w_head, layers, x, v_hat, v_hat_prev, v_fresh, score, g, mask,
+                      active_idx, h, k_caches, v_caches)
+
+
+def hsa_step(ctx: Context, model: ModelBinding, i: int, sigma_i: float, sigma_next: float,
+             regroup: bool = True) -> None:
+    _check(ctx.ptr, load().hsa_step(ctx.ptr, ctypes.byref(model.weights), ctypes.byref(model.state),
+                                    i, float(sigma_i), float(sigma_next), 1 if regroup else 0))

@@ -1,0 +1,95 @@
+// internal.h - context layout and kernel launchers shared by the .cu files of libhsa.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "../../include/hsa.h"
+
+namespace hsa {
+
+constexpr int kMaxGroups = 8;
+
+// Bits a kernel can set in the context's device flag (read by hsa_sync_check).
+enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_INDEX = 2, DEV_BAD_SCORE = 4, DEV_BAD_GROUP = 8 };
+constexpr int kRadixBins = 256;
+
+struct Ctx {
+  hsa_model_cfg cfg{};
+  int T = 0, K = 0, m = 0;
+  int budgets[kMaxGroups]{};
+  int counts[kMaxGroups]{};
+  int strides[kMaxGroups]{};
+  cudaStream_t stream = nullptr;
+  int device = 0;
+  int num_sms = 148;
+  std::string err;
+  // scratch (device)
+  void* u = nullptr;      // bf16 [N, D] LN output of the active rows
+  void* q = nullptr;      // bf16 [N, D] compact queries
+  void* o = nullptr;      // bf16 [N, D] compact attention output
+  void* hmid = nullptr;   // bf16 [N, F] compact MLP hidden
+  uint32_t* cuts = nullptr;  // selector cut keys, 2 words per cut
+  int* flag = nullptr;       // device error flag
+};
+
+// Row-index guard used by kernels that follow idx: out-of-range rows are
+// skipped and reported through the device flag.
+__device__ __forceinline__ bool row_ok(int32_t r, int N, int* flag) {
+  if (static_cast<uint32_t>(r) < static_cast<uint32_t>(N)) return true;
+  atomicOr(flag, DEV_BAD_INDEX);
+  return false;
+}
+
+// ---- launchers (return cudaGetLastError() of the launch)
+cudaError_t launch_schedule(const Ctx& c, int i, const uint8_t* g, uint8_t* mask, int32_t* idx,
+                            int32_t* n_dev);
+cudaError_t launch_score(const Ctx& c, const float* v_prev, const float* v_cur, float* score);
+cudaError_t launch_select(const Ctx& c, const float* score, uint8_t* g);
+cudaError_t launch_euler(const Ctx& c, float* x, float* v_hat, float* v_hat_prev,
+                         const float* v_fresh, const uint8_t* mask, float s0, float s1);
+cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, int n, void* u);
+cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_rows,
+                              const int32_t* idx, int n, void* kc, void* vc);
+cudaError_t launch_embed(const Ctx& c, const float* w_in, const float* x_lat, const int32_t* idx,
+                         int n, float* h);
+cudaError_t launch_head(const Ctx& c, const float* w_head, const float* h, const int32_t* idx,
+                        int n, float* v_fresh);
+
+// GEMM epilogues: C[m, j] = sum_k A[m, k] * B[j, k]  (A [M, K], B [Ncols, K], both bf16).
+enum GemmEpi : int {
+  EPI_STORE = 0,  // out bf16 [M, Ncols]
+  EPI_QKV = 1,    // Q -> out [M, D]; K, V -> caches rows idx[m]
+  EPI_RESID = 2,  // x[idx[m], j] += C  (fp32)
+  EPI_GELU = 3,   // out bf16 [M, Ncols] = GELU(C)
+};
+
+struct GemmArgs {
+  const void* A;   // bf16 [M, Kd]
+  const void* B;   // bf16 [Ncols, Kd]
+  int M, Ncols, Kd;
+  int epi;
+  void* out;          // EPI_STORE / EPI_GELU / EPI_QKV (Q)
+  int ld_out;         // elements
+  void* k_cache;      // EPI_QKV
+  void* v_cache;      // EPI_QKV
+  float* x;           // EPI_RESID
+  int ld_x;
+  const int32_t* idx; // EPI_QKV / EPI_RESID
+  int N;              // rows of caches / x (bounds for idx)
+};
+
+cudaError_t launch_gemm(const Ctx& c, const GemmArgs& a, std::string* why);
+
+cudaError_t launch_attention(const Ctx& c, const void* q, int n, const void* kc, const void* vc,
+                             void* o, std::string* why);
+
+// TMA descriptor for a row-major bf16 matrix [rows, cols] with a
+// box of [box_rows, 64] and 128-byte swizzle.  Returns false on failure.
+bool make_tmap_bf16(CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint64_t row_stride_elems, uint32_t box_rows, std::string* why);
+
+}  // namespace hsa

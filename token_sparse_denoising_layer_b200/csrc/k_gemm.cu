@@ -1,0 +1,283 @@
+// k_gemm.cu - active-row GEMMs of the HSA layer on the 5th-generation tensor
+// cores (tcgen05.mma, fp32 accumulators in TMEM, operands staged by TMA).
+//
+// C[m, j] = sum_k A[m, k] * B[j, k], A = compact bf16 activations of the
+// active rows [M = |A_i|, K], B = a Linear weight [Ncols, K].  The epilogue
+// is where the sparse structure of the method lives ("Technical Summary:
+// Heterogeneous Step Allocation (HSA) for Efficient Video Generation",
+// section 2.2): fresh K/V rows are scattered into the KV cache rows idx[m],
+// and out-projection / MLP results are added into residual rows idx[m].
+//
+// CTA tile 128 x BN (BN = 256 or 128), K-block 64, a multi-stage TMA ring.
+// Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs (one thread),
+// warps 2..5 drain TMEM and run the epilogue.
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace hsa {
+
+namespace {
+
+constexpr int kBM = 128;
+constexpr int kBK = 64;
+constexpr int kGemmThreads = 192;
+
+template <int BN>
+struct GemmCfg {
+  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kABytes = kBM * kBK * 2;
+  static constexpr int kBBytes = BN * kBK * 2;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kBarBytes = 256;
+  static constexpr int kSmem = kStages * kStageBytes + kBarBytes + 1024;
+};
+
+struct EpiParams {
+  int M, Ncols, Kd, epi;
+  __nv_bfloat16* out;
+  int ld_out;
+  __nv_bfloat16* kc;
+  __nv_bfloat16* vc;
+  float* x;
+  int ld_x;
+  const int32_t* idx;
+  int N;
+  int* flag;
+};
+
+__device__ __forceinline__ float gelu_f(float v) {
+  return 0.5f * v * (1.0f + erff(v * 0.70710678118654752440f));
+}
+
+// 32 fp32 accumulators -> 32 bf16 at dst (64 contiguous bytes, 16-byte aligned).
+template <bool kGelu>
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t (&r)[32]) {
+  uint4* d4 = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    uint32_t w[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      float a = __uint_as_float(r[8 * v + 2 * e]);
+      float b = __uint_as_float(r[8 * v + 2 * e + 1]);
+      if (kGelu) {
+        a = gelu_f(a);
+        b = gelu_f(b);
+      }
+      w[e] = pack_bf16(a, b);
+    }
+    d4[v] = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+}
+
+// x[dst .. dst+31] += r (fp32, 128 contiguous bytes).
+__device__ __forceinline__ void add_f32x32(float* dst, const uint32_t (&r)[32]) {
+  float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+  for (int v = 0; v < 8; ++v) {
+    float4 a = d4[v];
+    a.x += __uint_as_float(r[4 * v]);
+    a.y += __uint_as_float(r[4 * v + 1]);
+    a.z += __uint_as_float(r[4 * v + 2]);
+    a.w += __uint_as_float(r[4 * v + 3]);
+    d4[v] = a;
+  }
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+           EpiParams p) {
+  using Cfg = GemmCfg<BN>;
+  constexpr int S = Cfg::kStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * Cfg::kABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * Cfg::kBBytes);
+  uint64_t* empty = full + S;
+  uint64_t* accf = empty + S;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
+  const int nk = p.Kd / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(accf, 1);
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, BN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int issued = 0;
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (kb / S) & 1;
+        if (!mbar_wait(&empty[s], ph ^ 1)) {
+          ok = false;
+          break;
+        }
+        mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
+        tma_load_2d(sA + s * Cfg::kABytes, &tmA, &full[s], kb * kBK, m0);
+        tma_load_2d(sB + s * Cfg::kBBytes, &tmB, &full[s], kb * kBK, n0);
+        issued = kb + 1;
+      }
+      if (!ok) {  // let copies already in flight land before the CTA exits
+        for (int kb = issued > S ? issued - S : 0; kb < issued; ++kb)
+          (void)mbar_wait(&full[kb % S], (kb / S) & 1);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_bf16(kBM, BN, false, false);
+      for (int kb = 0; kb < nk; ++kb) {
+        const int s = kb % S;
+        const uint32_t ph = (kb / S) & 1;
+        if (!mbar_wait(&full[s], ph)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t a0 = smem_u32(sA + s * Cfg::kABytes);
+        const uint32_t b0 = smem_u32(sB + s * Cfg::kBBytes);
+#pragma unroll
+        for (int kk = 0; kk < kBK / 16; ++kk) {
+          const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+          const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
+          umma_bf16(tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&empty[s]);
+      }
+      umma_commit(accf);
+    }
+  } else {
+    // epilogue: warp w reads TMEM lanes [32*(w%4), +32) = tile rows
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const int m = m0 + row;
+    const bool waited = __all_sync(0xffffffffu, mbar_wait(accf, 0));
+    if (!waited) {
+      ok = false;
+    } else {
+      tc_fence_after();
+      const bool mrow = m < p.M;
+      int32_t dst_row = 0;
+      if (mrow && (p.epi == EPI_QKV || p.epi == EPI_RESID)) {
+        dst_row = __ldg(p.idx + m);
+        if (!row_ok(dst_row, p.N, p.flag)) dst_row = -1;
+      }
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16);
+#pragma unroll 1
+      for (int c0 = 0; c0 < BN; c0 += 32) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld32(tbase + c0, r);
+        const int col = n0 + c0;
+        if (mrow && col < p.Ncols) switch (p.epi) {
+          case EPI_STORE:
+            store_bf16x32<false>(p.out + static_cast<size_t>(m) * p.ld_out + col, r);
+            break;
+          case EPI_GELU:
+            store_bf16x32<true>(p.out + static_cast<size_t>(m) * p.ld_out + col, r);
+            break;
+          case EPI_QKV: {
+            const int D = p.ld_out;
+            const int which = col / D;
+            const int cc = col - which * D;
+            if (which == 0) {
+              store_bf16x32<false>(p.out + static_cast<size_t>(m) * D + cc, r);
+            } else if (dst_row >= 0) {
+              __nv_bfloat16* cache = which == 1 ? p.kc : p.vc;
+              store_bf16x32<false>(cache + static_cast<size_t>(dst_row) * D + cc, r);
+            }
+            break;
+          }
+          case EPI_RESID:
+            if (dst_row >= 0) add_f32x32(p.x + static_cast<size_t>(dst_row) * p.ld_x + col, r);
+            break;
+          default:
+            break;
+        }
+      }
+    }
+  }
+  if (!ok) atomicOr(p.flag, DEV_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, BN);
+  }
+}
+
+template <int BN>
+cudaError_t launch_bn(const Ctx& c, const GemmArgs& a, std::string* why) {
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16(&ta, a.A, a.M, a.Kd, a.Kd, kBM, why)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&tb, a.B, a.Ncols, a.Kd, a.Kd, BN, why)) return cudaErrorInvalidValue;
+  EpiParams p{};
+  p.M = a.M;
+  p.Ncols = a.Ncols;
+  p.Kd = a.Kd;
+  p.epi = a.epi;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.ld_out = a.ld_out;
+  p.kc = static_cast<__nv_bfloat16*>(a.k_cache);
+  p.vc = static_cast<__nv_bfloat16*>(a.v_cache);
+  p.x = a.x;
+  p.ld_x = a.ld_x;
+  p.idx = a.idx;
+  p.N = a.N;
+  p.flag = c.flag;
+  constexpr int smem = GemmCfg<BN>::kSmem;
+  static bool attr_set = false;  // one device per process is the supported use
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const dim3 grid((a.Ncols + BN - 1) / BN, (a.M + kBM - 1) / kBM);
+  k_gemm<BN><<<grid, kGemmThreads, smem, c.stream>>>(ta, tb, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const Ctx& c, const GemmArgs& a, std::string* why) {
+  if (a.M <= 0) return cudaSuccess;
+  if (a.Kd % kBK != 0 || a.Ncols % 32 != 0) {
+    if (why) *why = "GEMM needs K % 64 == 0 and Ncols % 32 == 0";
+    return cudaErrorInvalidValue;
+  }
+  if (a.Ncols % 256 == 0) return launch_bn<256>(c, a, why);
+  return launch_bn<128>(c, a, why);
+}
+
+}  // namespace hsa

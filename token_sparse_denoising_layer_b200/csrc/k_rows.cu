@@ -1,0 +1,275 @@
+// k_rows.cu - row kernels around the active-only forward of the HSA step:
+// LayerNorm gather of the active rows, the standalone KV-cache scatter, the
+// latent embed of the active rows and the velocity head.
+//
+// Method: "Technical Summary: Heterogeneous Step Allocation (HSA) for
+// Efficient Video Generation", section 2.2 (KV-Cache Synchronization): only
+// the active tokens A_i are processed, and their fresh K/V rows overwrite the
+// stale rows of the per-layer cache.
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace hsa {
+
+constexpr float kLnEps = 1e-5f;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// Mean and reciprocal standard deviation of a row held as NCH float4 per lane
+// (the row is 128*NCH wide); two passes over registers.
+template <int NCH>
+__device__ __forceinline__ void row_stats(const float4 (&v)[NCH], int D, float& mean, float& rstd) {
+  float s = 0.f;
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) s += (v[c].x + v[c].y) + (v[c].z + v[c].w);
+  mean = warp_sum(s) / static_cast<float>(D);
+  float q = 0.f;
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    const float a = v[c].x - mean, b = v[c].y - mean, e = v[c].z - mean, f = v[c].w - mean;
+    q += (a * a + b * b) + (e * e + f * f);
+  }
+  const float var = warp_sum(q) / static_cast<float>(D);
+  rstd = 1.0f / sqrtf(var + kLnEps);
+}
+
+// ------------------------------------------------------------ LN gather
+// One warp per active row: u[m] = bf16(LN(x[idx[m]])).  D = 128 * NCH.
+template <int NCH>
+__global__ void __launch_bounds__(256) k_ln_gather(const float* __restrict__ x,
+                                                   const int32_t* __restrict__ idx, int n, int N,
+                                                   __nv_bfloat16* __restrict__ u, int* flag) {
+  const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (m >= n) return;
+  constexpr int D = 128 * NCH;
+  const int r = __ldg(idx + m);
+  uint2* out = reinterpret_cast<uint2*>(u + static_cast<size_t>(m) * D);
+  if (!row_ok(r, N, flag)) {
+#pragma unroll
+    for (int c = 0; c < NCH; ++c) out[c * 32 + lane] = make_uint2(0u, 0u);
+    return;
+  }
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(r) * D);
+  float4 v[NCH];
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) v[c] = __ldg(xr + c * 32 + lane);
+  float mean, rstd;
+  row_stats<NCH>(v, D, mean, rstd);
+#pragma unroll
+  for (int c = 0; c < NCH; ++c) {
+    const uint32_t lo = pack_bf16((v[c].x - mean) * rstd, (v[c].y - mean) * rstd);
+    const uint32_t hi = pack_bf16((v[c].z - mean) * rstd, (v[c].w - mean) * rstd);
+    out[c * 32 + lane] = make_uint2(lo, hi);
+  }
+}
+
+// Any D multiple of 128: three passes over the row (L1/L2 serve the re-reads).
+__global__ void __launch_bounds__(256) k_ln_gather_any(const float* __restrict__ x,
+                                                       const int32_t* __restrict__ idx, int n,
+                                                       int N, int D,
+                                                       __nv_bfloat16* __restrict__ u, int* flag) {
+  const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (m >= n) return;
+  const int r = __ldg(idx + m);
+  uint2* out = reinterpret_cast<uint2*>(u + static_cast<size_t>(m) * D);
+  const int nv = D / 4;
+  if (!row_ok(r, N, flag)) {
+    for (int c = lane; c < nv; c += 32) out[c] = make_uint2(0u, 0u);
+    return;
+  }
+  const float4* xr = reinterpret_cast<const float4*>(x + static_cast<size_t>(r) * D);
+  float s = 0.f;
+  for (int c = lane; c < nv; c += 32) {
+    const float4 a = __ldg(xr + c);
+    s += (a.x + a.y) + (a.z + a.w);
+  }
+  const float mean = warp_sum(s) / static_cast<float>(D);
+  float q = 0.f;
+  for (int c = lane; c < nv; c += 32) {
+    const float4 a = __ldg(xr + c);
+    const float p0 = a.x - mean, p1 = a.y - mean, p2 = a.z - mean, p3 = a.w - mean;
+    q += (p0 * p0 + p1 * p1) + (p2 * p2 + p3 * p3);
+  }
+  const float rstd = 1.0f / sqrtf(warp_sum(q) / static_cast<float>(D) + kLnEps);
+  for (int c = lane; c < nv; c += 32) {
+    const float4 a = __ldg(xr + c);
+    out[c] = make_uint2(pack_bf16((a.x - mean) * rstd, (a.y - mean) * rstd),
+                        pack_bf16((a.z - mean) * rstd, (a.w - mean) * rstd));
+  }
+}
+
+cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, int n, void* u) {
+  if (n <= 0) return cudaSuccess;
+  const int D = c.cfg.D, N = c.cfg.N;
+  const dim3 grid((n + 7) / 8), block(256);
+  auto* uo = static_cast<__nv_bfloat16*>(u);
+  switch (D / 128) {
+    case 1: k_ln_gather<1><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
+    case 2: k_ln_gather<2><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
+    case 4: k_ln_gather<4><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
+    case 8: k_ln_gather<8><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
+    case 12: k_ln_gather<12><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
+    case 16: k_ln_gather<16><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
+    default: k_ln_gather_any<<<grid, block, 0, c.stream>>>(x, idx, n, N, D, uo, c.flag); break;
+  }
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ KV scatter
+// k_cache[idx[m]] = k_rows[m], v_cache[idx[m]] = v_rows[m]; 16-byte vectors.
+__global__ void __launch_bounds__(256) k_kv_scatter(const uint4* __restrict__ k_rows,
+                                                    const uint4* __restrict__ v_rows,
+                                                    const int32_t* __restrict__ idx, int n, int N,
+                                                    int vec_per_row, uint4* __restrict__ kc,
+                                                    uint4* __restrict__ vc, int* flag) {
+  const size_t total = static_cast<size_t>(n) * vec_per_row;
+  for (size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; t < total;
+       t += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int m = static_cast<int>(t / vec_per_row);
+    const int c = static_cast<int>(t - static_cast<size_t>(m) * vec_per_row);
+    const int r = __ldg(idx + m);
+    if (!row_ok(r, N, flag)) continue;
+    const size_t dst = static_cast<size_t>(r) * vec_per_row + c;
+    __stcs(kc + dst, __ldcs(k_rows + t));
+    __stcs(vc + dst, __ldcs(v_rows + t));
+  }
+}
+
+cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_rows,
+                              const int32_t* idx, int n, void* kc, void* vc) {
+  if (n <= 0) return cudaSuccess;
+  const int vpr = c.cfg.D / 8;
+  const size_t total = static_cast<size_t>(n) * vpr;
+  size_t blocks = (total + 255) / 256;
+  const size_t cap = static_cast<size_t>(c.num_sms) * 16;
+  if (blocks > cap) blocks = cap;
+  k_kv_scatter<<<static_cast<unsigned>(blocks), 256, 0, c.stream>>>(
+      static_cast<const uint4*>(k_rows), static_cast<const uint4*>(v_rows), idx, n, c.cfg.N, vpr,
+      static_cast<uint4*>(kc), static_cast<uint4*>(vc), c.flag);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ embed
+// h[idx[m], j] = sum_c W_in[j, c] * x_lat[idx[m], c]; C = 16, four j per thread.
+__global__ void __launch_bounds__(256) k_embed(const float* __restrict__ w_in,
+                                               const float* __restrict__ x_lat,
+                                               const int32_t* __restrict__ idx, int n, int N,
+                                               int D, float* __restrict__ h, int* flag) {
+  const int q4 = D / 4;
+  const size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (t >= static_cast<size_t>(n) * q4) return;
+  const int m = static_cast<int>(t / q4);
+  const int j0 = static_cast<int>(t - static_cast<size_t>(m) * q4) * 4;
+  const int r = __ldg(idx + m);
+  if (!row_ok(r, N, flag)) return;
+  const float4* xl = reinterpret_cast<const float4*>(x_lat + static_cast<size_t>(r) * 16);
+  float xv[16];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 a = __ldg(xl + q);
+    xv[4 * q] = a.x;
+    xv[4 * q + 1] = a.y;
+    xv[4 * q + 2] = a.z;
+    xv[4 * q + 3] = a.w;
+  }
+  float acc[4];
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+    const float4* wr = reinterpret_cast<const float4*>(w_in + static_cast<size_t>(j0 + jj) * 16);
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 w = __ldg(wr + q);
+      s = fmaf(w.x, xv[4 * q], s);
+      s = fmaf(w.y, xv[4 * q + 1], s);
+      s = fmaf(w.z, xv[4 * q + 2], s);
+      s = fmaf(w.w, xv[4 * q + 3], s);
+    }
+    acc[jj] = s;
+  }
+  *reinterpret_cast<float4*>(h + static_cast<size_t>(r) * D + j0) =
+      make_float4(acc[0], acc[1], acc[2], acc[3]);
+}
+
+cudaError_t launch_embed(const Ctx& c, const float* w_in, const float* x_lat, const int32_t* idx,
+                         int n, float* h) {
+  if (n <= 0) return cudaSuccess;
+  const size_t total = static_cast<size_t>(n) * (c.cfg.D / 4);
+  k_embed<<<static_cast<unsigned>((total + 255) / 256), 256, 0, c.stream>>>(
+      w_in, x_lat, idx, n, c.cfg.N, c.cfg.D, h, c.flag);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------ velocity head
+// One warp per active row: v_fresh[idx[m], o] = sum_j LN(h[idx[m]])_j W_head[o, j].
+// fp32 throughout; the 16 dot products are reduced with butterflies.
+__global__ void __launch_bounds__(256) k_head(const float* __restrict__ w_head,
+                                              const float* __restrict__ h,
+                                              const int32_t* __restrict__ idx, int n, int N,
+                                              int D, float* __restrict__ v_fresh, int* flag) {
+  const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (m >= n) return;
+  const int r = __ldg(idx + m);
+  if (!row_ok(r, N, flag)) return;
+  const float4* hr = reinterpret_cast<const float4*>(h + static_cast<size_t>(r) * D);
+  const int nv = D / 4;
+  float s = 0.f;
+  for (int c = lane; c < nv; c += 32) {
+    const float4 a = __ldg(hr + c);
+    s += (a.x + a.y) + (a.z + a.w);
+  }
+  const float mean = warp_sum(s) / static_cast<float>(D);
+  float q = 0.f;
+  for (int c = lane; c < nv; c += 32) {
+    const float4 a = __ldg(hr + c);
+    const float p0 = a.x - mean, p1 = a.y - mean, p2 = a.z - mean, p3 = a.w - mean;
+    q += (p0 * p0 + p1 * p1) + (p2 * p2 + p3 * p3);
+  }
+  const float rstd = 1.0f / sqrtf(warp_sum(q) / static_cast<float>(D) + kLnEps);
+  float acc[16];
+#pragma unroll
+  for (int o = 0; o < 16; ++o) acc[o] = 0.f;
+  for (int c = lane; c < nv; c += 32) {
+    float4 a = __ldg(hr + c);
+    a.x = (a.x - mean) * rstd;
+    a.y = (a.y - mean) * rstd;
+    a.z = (a.z - mean) * rstd;
+    a.w = (a.w - mean) * rstd;
+#pragma unroll
+    for (int o = 0; o < 16; ++o) {
+      const float4 w = __ldg(reinterpret_cast<const float4*>(w_head + static_cast<size_t>(o) * D) + c);
+      acc[o] = fmaf(a.x, w.x, fmaf(a.y, w.y, fmaf(a.z, w.z, fmaf(a.w, w.w, acc[o]))));
+    }
+  }
+#pragma unroll
+  for (int o = 0; o < 16; ++o) acc[o] = warp_sum(acc[o]);
+  if (lane < 4) {
+    // lane l writes channels 4l..4l+3 (constant register indices)
+    float4 outv = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int l = 0; l < 4; ++l)
+      if (lane == l) outv = make_float4(acc[4 * l], acc[4 * l + 1], acc[4 * l + 2], acc[4 * l + 3]);
+    reinterpret_cast<float4*>(v_fresh + static_cast<size_t>(r) * 16)[lane] = outv;
+  }
+}
+
+cudaError_t launch_head(const Ctx& c, const float* w_head, const float* h, const int32_t* idx,
+                        int n, float* v_fresh) {
+  if (n <= 0) return cudaSuccess;
+  k_head<<<(n + 7) / 8, 256, 0, c.stream>>>(w_head, h, idx, n, c.cfg.N, c.cfg.D, v_fresh, c.flag);
+  return cudaGetLastError();
+}
+
+}  // namespace hsa

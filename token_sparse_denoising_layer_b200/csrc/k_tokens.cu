@@ -1,0 +1,359 @@
+// k_tokens.cu - per-token kernels of the HSA step: group schedule, L1
+// relative-change score, exact radix selection of the groups, and the
+// cached Euler update.
+//
+// Method: "Technical Summary: Heterogeneous Step Allocation (HSA) for
+// Efficient Video Generation", section 2.1 (Token Partitioning and
+// Scheduling, Dynamic Selection) and section 2.3 (Cached Euler Update).
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace hsa {
+
+// ============================================================ schedule (2.1)
+//
+// Token n of group k is active at iteration i iff i mod (T/s_k) == 0; in the
+// phase window (first/last m iterations, section 2.4) every token is active.
+// Each CTA owns a 4096-token chunk.  It counts the active tokens of all
+// earlier chunks itself (a read of at most N bytes from L2), so the compaction
+// needs one launch and no inter-CTA waiting.  Output order is ascending.
+
+constexpr int kSchedThreads = 1024;
+constexpr int kSchedChunk = kSchedThreads * 4;
+
+struct SchedParams {
+  int strides[kMaxGroups];
+  int K, i, T, m, N;
+};
+
+__device__ __forceinline__ uint32_t active_group_bits(const SchedParams& p) {
+  const bool window = p.m > 0 && (p.i < p.m || p.i >= p.T - p.m);
+  uint32_t bits = 0;
+  for (int k = 0; k < p.K; ++k)
+    if (window || (p.i % p.strides[k]) == 0) bits |= 1u << k;
+  return bits;
+}
+
+__device__ __forceinline__ int on_of(uint32_t gbyte, uint32_t bits) {
+  return gbyte < 32u ? static_cast<int>((bits >> gbyte) & 1u) : 0;
+}
+
+__device__ __forceinline__ int count_on_word(uint32_t w, uint32_t bits) {
+  return on_of(w & 0xFF, bits) + on_of((w >> 8) & 0xFF, bits) + on_of((w >> 16) & 0xFF, bits) +
+         on_of(w >> 24, bits);
+}
+
+// Block-wide exclusive scan of one int per thread; returns the exclusive
+// prefix and writes the block total to *total.
+__device__ __forceinline__ int block_exclusive_scan(int v, int* warp_sums, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) warp_sums[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = blockDim.x >> 5;
+    int s = lane < nw ? warp_sums[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      int y = __shfl_up_sync(0xffffffffu, s, o);
+      if (lane >= o) s += y;
+    }
+    if (lane < nw) warp_sums[lane] = s;  // inclusive
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? warp_sums[warp - 1] : 0) + x - v;
+  *total = warp_sums[(blockDim.x >> 5) - 1];
+  __syncthreads();
+  return before;
+}
+
+__device__ __forceinline__ int block_sum(int v, int* warp_sums) {
+  int total;
+  block_exclusive_scan(v, warp_sums, &total);
+  return total;
+}
+
+__global__ void __launch_bounds__(kSchedThreads) k_schedule(const uint8_t* __restrict__ g,
+                                                            uint8_t* __restrict__ mask,
+                                                            int32_t* __restrict__ idx,
+                                                            int32_t* __restrict__ n_dev,
+                                                            SchedParams p, int* flag) {
+  __shared__ int warp_sums[32];
+  const uint32_t bits = active_group_bits(p);
+  const int base = blockIdx.x * kSchedChunk;
+
+  // 1. active tokens before this chunk (base is a multiple of 16)
+  int before = 0;
+  const uint4* gv = reinterpret_cast<const uint4*>(g);
+  for (int v = threadIdx.x; v < base / 16; v += blockDim.x) {
+    const uint4 w = __ldg(gv + v);
+    before += count_on_word(w.x, bits) + count_on_word(w.y, bits) + count_on_word(w.z, bits) +
+              count_on_word(w.w, bits);
+  }
+  before = block_sum(before, warp_sums);
+
+  // 2. this thread's four tokens
+  const int n0 = base + 4 * threadIdx.x;
+  int on[4] = {0, 0, 0, 0};
+  int bad = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int n = n0 + j;
+    if (n < p.N) {
+      const uint32_t gb = g[n];
+      if (gb >= static_cast<uint32_t>(p.K)) bad = 1;
+      else on[j] = on_of(gb, bits);
+    }
+  }
+  if (bad) atomicOr(flag, DEV_BAD_GROUP);
+  const int mine = on[0] + on[1] + on[2] + on[3];
+  int total;
+  int pos = before + block_exclusive_scan(mine, warp_sums, &total);
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int n = n0 + j;
+    if (n < p.N) {
+      mask[n] = static_cast<uint8_t>(on[j]);
+      if (on[j]) idx[pos++] = n;
+    }
+  }
+  if (n_dev != nullptr && threadIdx.x == 0 && base + kSchedChunk >= p.N) *n_dev = before + total;
+}
+
+cudaError_t launch_schedule(const Ctx& c, int i, const uint8_t* g, uint8_t* mask, int32_t* idx,
+                            int32_t* n_dev) {
+  SchedParams p{};
+  for (int k = 0; k < c.K; ++k) p.strides[k] = c.strides[k];
+  p.K = c.K;
+  p.i = i;
+  p.T = c.T;
+  p.m = c.m;
+  p.N = c.cfg.N;
+  const int blocks = (c.cfg.N + kSchedChunk - 1) / kSchedChunk;
+  k_schedule<<<blocks, kSchedThreads, 0, c.stream>>>(g, mask, idx, n_dev, p, c.flag);
+  return cudaGetLastError();
+}
+
+// ============================================================ selector (2.1)
+//
+// Score: r_n = sum_c |v_cur - v_prev| / (sum_c |v_prev| + 1e-6) in float32,
+// channel order, explicit round-to-nearest operations (no contraction), so
+// the value is reproducible bit for bit.
+
+constexpr float kScoreEps = 1e-6f;
+
+__global__ void __launch_bounds__(256) k_score(const float4* __restrict__ v_prev,
+                                               const float4* __restrict__ v_cur,
+                                               float* __restrict__ score, int N, int* flag) {
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  float num = 0.f, den = 0.f;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 a = __ldg(v_prev + 4 * n + q);
+    const float4 b = __ldg(v_cur + 4 * n + q);
+    num = __fadd_rn(num, fabsf(__fsub_rn(b.x, a.x)));
+    den = __fadd_rn(den, fabsf(a.x));
+    num = __fadd_rn(num, fabsf(__fsub_rn(b.y, a.y)));
+    den = __fadd_rn(den, fabsf(a.y));
+    num = __fadd_rn(num, fabsf(__fsub_rn(b.z, a.z)));
+    den = __fadd_rn(den, fabsf(a.z));
+    num = __fadd_rn(num, fabsf(__fsub_rn(b.w, a.w)));
+    den = __fadd_rn(den, fabsf(a.w));
+  }
+  den = __fadd_rn(den, kScoreEps);
+  const float r = __fadd_rn(__fdiv_rn(num, den), 0.0f);
+  if (!(r >= 0.f) || isinf(r)) atomicOr(flag, DEV_BAD_SCORE);
+  score[n] = r;
+}
+
+cudaError_t launch_score(const Ctx& c, const float* v_prev, const float* v_cur, float* score) {
+  const int N = c.cfg.N;
+  k_score<<<(N + 255) / 256, 256, 0, c.stream>>>(reinterpret_cast<const float4*>(v_prev),
+                                                 reinterpret_cast<const float4*>(v_cur), score, N,
+                                                 c.flag);
+  return cudaGetLastError();
+}
+
+// Ranking key: tokens sorted by (score descending, index ascending) are the
+// tokens sorted by the 64-bit key (~bits(score), n) ascending.  For finite
+// non-negative floats the bit pattern is monotone in the value.
+__device__ __forceinline__ uint32_t key_hi(float r) { return ~__float_as_uint(__fadd_rn(r, 0.0f)); }
+
+// One CTA per cut j: find the key of rank R_j (0-based), where
+// R_j = n_1 + ... + n_j.  Four 8-bit radix passes fix the high word exactly;
+// the index tie-break is then the (R_j - count(hi < hv))-th token, in index
+// order, among those whose high word equals hv.  Only integer shared-memory
+// atomics are used, so the result is deterministic.
+constexpr int kSelThreads = 1024;
+
+struct CutParams {
+  int rank[kMaxGroups];
+};
+
+__global__ void __launch_bounds__(kSelThreads) k_radix_cut(const float* __restrict__ score, int N,
+                                                           CutParams cp, uint32_t* cuts,
+                                                           int* flag) {
+  __shared__ int hist[kRadixBins];
+  __shared__ int warp_sums[32];
+  __shared__ uint32_t s_sel[2];
+  const int j = blockIdx.x;
+  const int R = cp.rank[j];
+  if (R >= N) {  // empty tail groups: a cut no key reaches
+    if (threadIdx.x == 0) {
+      cuts[2 * j] = 0xFFFFFFFFu;
+      cuts[2 * j + 1] = 0xFFFFFFFFu;
+    }
+    return;
+  }
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = R;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int b = threadIdx.x; b < kRadixBins; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+    for (int n = threadIdx.x; n < N; n += blockDim.x) {
+      const float r = __ldg(score + n);
+      if (pass == 0 && !(r >= 0.f)) atomicOr(flag, DEV_BAD_SCORE);
+      const uint32_t h = key_hi(r);
+      if ((h & pmask) == prefix) atomicAdd(&hist[(h >> shift) & 0xFF], 1);
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // lane l owns bins 8l..8l+7
+      const int lane = threadIdx.x;
+      int loc[8];
+      int s = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        loc[t] = hist[8 * lane + t];
+        s += loc[t];
+      }
+      int incl = s;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int cum = incl - s;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (cum <= remaining && remaining < cum + loc[t]) {
+          s_sel[0] = static_cast<uint32_t>(8 * lane + t);
+          s_sel[1] = static_cast<uint32_t>(cum);
+        }
+        cum += loc[t];
+      }
+    }
+    __syncthreads();
+    const uint32_t bin = s_sel[0];
+    remaining -= static_cast<int>(s_sel[1]);
+    prefix |= bin << shift;
+    pmask |= 0xFFu << shift;
+    __syncthreads();
+  }
+  // tie-break by index: the remaining-th token (0-based) with key_hi == prefix
+  int running = 0;
+  for (int base = 0; base < N; base += blockDim.x) {
+    const int n = base + threadIdx.x;
+    const int eq = (n < N && key_hi(__ldg(score + n)) == prefix) ? 1 : 0;
+    int total;
+    const int pos = running + block_exclusive_scan(eq, warp_sums, &total);
+    if (eq && pos == remaining) {
+      cuts[2 * j] = prefix;
+      cuts[2 * j + 1] = static_cast<uint32_t>(n);
+    }
+    running += total;
+    if (running > remaining) break;  // uniform across the block
+  }
+}
+
+__global__ void __launch_bounds__(256) k_assign(const float* __restrict__ score,
+                                                const uint32_t* __restrict__ cuts, int ncut,
+                                                uint8_t* __restrict__ g, int N) {
+  __shared__ uint32_t s_cut[2 * kMaxGroups];
+  if (threadIdx.x < 2 * ncut) s_cut[threadIdx.x] = cuts[threadIdx.x];
+  __syncthreads();
+  const int n = blockIdx.x * blockDim.x + threadIdx.x;
+  if (n >= N) return;
+  const uint32_t h = key_hi(__ldg(score + n));
+  uint32_t k = 0;
+  for (int j = 0; j < ncut; ++j) {
+    const uint32_t ch = s_cut[2 * j], ci = s_cut[2 * j + 1];
+    k += (h > ch || (h == ch && static_cast<uint32_t>(n) >= ci)) ? 1u : 0u;
+  }
+  g[n] = static_cast<uint8_t>(k);
+}
+
+cudaError_t launch_select(const Ctx& c, const float* score, uint8_t* g) {
+  const int N = c.cfg.N;
+  const int ncut = c.K - 1;
+  if (ncut == 0) {
+    cudaError_t e = cudaMemsetAsync(g, 0, static_cast<size_t>(N), c.stream);
+    return e;
+  }
+  CutParams cp{};
+  int acc = 0;
+  for (int j = 0; j < ncut; ++j) {
+    acc += c.counts[j];
+    cp.rank[j] = acc;
+  }
+  k_radix_cut<<<ncut, kSelThreads, 0, c.stream>>>(score, N, cp, c.cuts, c.flag);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_assign<<<(N + 255) / 256, 256, 0, c.stream>>>(score, c.cuts, ncut, g, N);
+  return cudaGetLastError();
+}
+
+// ============================================================ cached Euler (2.3)
+//
+// One pass over all N tokens, four channels per thread (128-bit accesses):
+// active tokens rotate their velocity cache (v_hat_prev <- v_hat <- v_fresh),
+// then every token advances by (sigma_next - sigma_i) * v_hat.  Inactive
+// tokens read neither v_fresh nor write the caches (predicated, not branched
+// per warp).  Float32 with one rounding per operation.
+
+__global__ void __launch_bounds__(256) k_euler(float4* __restrict__ x, float4* __restrict__ v_hat,
+                                               float4* __restrict__ v_hat_prev,
+                                               const float4* __restrict__ v_fresh,
+                                               const uint8_t* __restrict__ mask, float s0,
+                                               float s1, int n4) {
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= n4) return;
+  const float d = __fsub_rn(s1, s0);
+  const bool on = __ldg(mask + (t >> 2)) != 0;
+  float4 h = __ldcs(v_hat + t);
+  float4 xx = __ldcs(x + t);
+  if (on) {
+    const float4 f = __ldcs(v_fresh + t);
+    __stcs(v_hat_prev + t, h);
+    __stcs(v_hat + t, f);
+    h = f;
+  }
+  xx.x = __fadd_rn(xx.x, __fmul_rn(d, h.x));
+  xx.y = __fadd_rn(xx.y, __fmul_rn(d, h.y));
+  xx.z = __fadd_rn(xx.z, __fmul_rn(d, h.z));
+  xx.w = __fadd_rn(xx.w, __fmul_rn(d, h.w));
+  __stcs(x + t, xx);
+}
+
+cudaError_t launch_euler(const Ctx& c, float* x, float* v_hat, float* v_hat_prev,
+                         const float* v_fresh, const uint8_t* mask, float s0, float s1) {
+  const int n4 = c.cfg.N * (c.cfg.C / 4);
+  k_euler<<<(n4 + 255) / 256, 256, 0, c.stream>>>(
+      reinterpret_cast<float4*>(x), reinterpret_cast<float4*>(v_hat),
+      reinterpret_cast<float4*>(v_hat_prev), reinterpret_cast<const float4*>(v_fresh), mask, s0,
+      s1, n4);
+  return cudaGetLastError();
+}
+
+}  // namespace hsa

@@ -228,3 +228,21 @@ def score_buffer(N: int, seed: int, n_tie_values: int = 0) -> np.ndarray:
         s = np.abs(r.standard_normal(N).astype(np.float32))
     s[r.integers(0, N, max(1, N // 100))] = 0.0
     return s.astype(np.float32)
+
+
+def device_layer_weights(D: int, F: int, seed: int, device="cuda"):
+    """Block weights ~ N(0, 1/fan_in) drawn on the device (torch Philox), bf16.
+
+    For workloads whose weights are too large to draw on the host quickly
+    (tens of layers at D = 1536).  Returns (w_qkv, w_o, w_1, w_2).
+    """
+    import torch
+
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+
+    def lin(o, i):
+        return (torch.randn((o, i), generator=g, device=device, dtype=torch.float32)
+                * (1.0 / np.sqrt(i))).to(torch.bfloat16)
+
+    return lin(3 * D, D), lin(D, D), lin(F, D), lin(D, F)
