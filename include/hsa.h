@@ -46,7 +46,8 @@ typedef enum {
   HSA_ERR_CUDA = 4,         /* a CUDA runtime/driver call failed */
   HSA_ERR_OOM = 5,          /* scratch allocation failed in hsa_create */
   HSA_ERR_TIMEOUT = 6,      /* a kernel's bounded wait expired (read by hsa_sync_check) */
-  HSA_ERR_DEVICE_CHECK = 7  /* a kernel found a bad index or a NaN score (hsa_sync_check) */
+  HSA_ERR_DEVICE_CHECK = 7, /* a kernel found a bad index or a NaN score (hsa_sync_check) */
+  HSA_ERR_SCRATCH_LIMIT = 8 /* a size beyond the fixed scratch of hsa_select_groups_static */
 } hsa_status;
 
 /* Model shape.  N tokens, C latent channels, D hidden, H heads, F MLP width, L layers. */
@@ -266,6 +267,33 @@ hsa_status hsa_euler_step(hsa_ctx* ctx, float* x, float* v_hat, float* v_hat_pre
  */
 hsa_status hsa_step(hsa_ctx* ctx, const hsa_model_weights* w, const hsa_state* s, int i,
                     float sigma_i, float sigma_next, int regroup);
+
+/*
+ * Group selection without any device allocation.  The paper has no
+ * counterpart: this is a service for callers that cannot call cudaMalloc,
+ * such as a host framework that owns all device memory through its own pool
+ * and forbids a library to allocate, or a latency-critical serving loop
+ * where cudaMalloc's implicit device synchronisation would stall other work.
+ *
+ * Same result as hsa_select_groups (scores, then exact group assignment with
+ * ties broken by token index), but it needs no context: the scores and cut
+ * keys live in one static device array of the library, sized for at most
+ * HSA_SELECT_STATIC_MAX_N tokens (512 KiB + 256 B), which every GPU that
+ * loads the library holds until the process exits.
+ *   v_prev, v_cur (device) fp32 [N, 16];  counts (host) n_1..n_K, sum == N;
+ *   g (device) uint8 [N] out;  stream cudaStream_t (NULL = legacy default).
+ * Returns HSA_ERR_SCRATCH_LIMIT when N > HSA_SELECT_STATIC_MAX_N, and the
+ * other argument errors of hsa_create / hsa_select_groups; there is no
+ * message string.  Calls no cudaMalloc or cudaFree.  The first call on a
+ * device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.
+ * All calls share the array and it keeps the last call's contents; calls
+ * that overlap on the GPU race on it.  Device-side checks (a NaN score) are
+ * not reported by this call.
+ */
+#define HSA_SELECT_STATIC_MAX_N 131072
+hsa_status hsa_select_groups_static(const float* v_prev, const float* v_cur, int N,
+                                    const int* counts, int K, uint8_t* g, void* stream);
 
 #ifdef __cplusplus
 }

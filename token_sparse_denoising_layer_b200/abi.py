@@ -21,11 +21,14 @@ SYMBOLS = [
     "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
     "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_linear", "hsa_kv_scatter",
     "hsa_attention", "hsa_out_proj_residual", "hsa_mlp_residual", "hsa_layer_forward",
-    "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_step",
+    "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_step", "hsa_select_groups_static",
 ]
 
 STATUS = {0: "HSA_OK", 1: "HSA_ERR_INVALID_ARG", 2: "HSA_ERR_BUDGET", 3: "HSA_ERR_SHAPE",
-          4: "HSA_ERR_CUDA", 5: "HSA_ERR_OOM", 6: "HSA_ERR_TIMEOUT", 7: "HSA_ERR_DEVICE_CHECK"}
+          4: "HSA_ERR_CUDA", 5: "HSA_ERR_OOM", 6: "HSA_ERR_TIMEOUT", 7: "HSA_ERR_DEVICE_CHECK",
+          8: "HSA_ERR_SCRATCH_LIMIT"}
+
+SELECT_STATIC_MAX_N = 131072  # HSA_SELECT_STATIC_MAX_N in include/hsa.h
 
 
 class HsaError(RuntimeError):
@@ -95,6 +98,7 @@ def load() -> ctypes.CDLL:
         "hsa_head": (I, [P, P, P, P, I, P]),
         "hsa_euler_step": (I, [P, P, P, P, P, P, F, F]),
         "hsa_step": (I, [P, ctypes.POINTER(hsa_model_weights), ctypes.POINTER(hsa_state), I, F, F, I]),
+        "hsa_select_groups_static": (I, [P, P, I, ctypes.POINTER(I), I, P, P]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -271,3 +275,17 @@ def hsa_step(ctx: Context, model: ModelBinding, i: int, sigma_i: float, sigma_ne
              regroup: bool = True) -> None:
     _check(ctx.ptr, load().hsa_step(ctx.ptr, ctypes.byref(model.weights), ctypes.byref(model.state),
                                     i, float(sigma_i), float(sigma_next), 1 if regroup else 0))
+
+
+def hsa_select_groups_static(v_prev, v_cur, N: int, counts: Sequence[int], g, stream=None) -> None:
+    """Group selection without a context or any device allocation (see include/hsa.h).
+
+    Its scratch is one static device array of the library, sized for at most
+    SELECT_STATIC_MAX_N tokens; concurrent calls on the GPU race on it.
+    """
+    K = len(counts)
+    c = (ctypes.c_int * K)(*counts)
+    st = load().hsa_select_groups_static(_p(v_prev), _p(v_cur), N, c, K, _p(g), _stream_ptr(stream))
+    if st != 0:
+        why = {8: f"N = {N} exceeds the static scratch limit of {SELECT_STATIC_MAX_N} tokens"}
+        raise HsaError(st, why.get(st, "hsa_select_groups_static rejected its arguments"))

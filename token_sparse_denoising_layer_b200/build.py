@@ -22,7 +22,7 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 BUILD = os.path.join(PKG, "_build")
 LIB = os.path.join(PKG, "libhsa.so")
-SOURCES = ["api.cu", "k_tokens.cu", "k_rows.cu", "k_gemm.cu", "k_attn.cu"]
+SOURCES = ["api.cu", "k_tokens.cu", "k_rows.cu", "k_gemm.cu", "k_attn.cu", "k_select_static.cu"]
 HEADERS = ["ptx.cuh", "internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xptxas", "-v",

@@ -1,0 +1,101 @@
+// k_select_static.cu - group selection that allocates no device memory.
+//
+// hsa_select_groups needs a context, and hsa_create allocates the context's
+// scratch with cudaMalloc.  Some callers cannot do that: a host framework
+// that owns every byte of device memory through its own pool and forbids a
+// library from allocating behind its back, or a latency-critical serving loop
+// where cudaMalloc's implicit device-wide synchronisation would stall other
+// streams.  hsa_select_groups_static gives them the same selection (scores,
+// exact radix cut search, group assignment) with its scratch -- the per-token
+// scores and the cut keys -- in one file-scope device array of fixed size.
+//
+// That array exists once per GPU that loads this library and stays allocated
+// until the process exits.  Every call shares it and it keeps the previous
+// call's contents; calls that overlap on the GPU (on two streams, or from two
+// threads) race on it.
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <mutex>
+#include <string>
+
+#include "../../include/hsa.h"
+#include "internal.h"
+
+namespace {
+
+constexpr int kStaticMaxN = HSA_SELECT_STATIC_MAX_N;
+constexpr size_t kScoreBytes = static_cast<size_t>(kStaticMaxN) * sizeof(float);
+constexpr size_t kCutBytes = 2 * hsa::kMaxGroups * sizeof(uint32_t);
+constexpr size_t kScratchBytes = kScoreBytes + kCutBytes + 256;
+
+// scores [kStaticMaxN] fp32 | cut keys [16] u32 | error flag (int) at an aligned offset
+static __device__ __align__(256) unsigned char g_select_scratch[kScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_setup_mutex;
+void* g_scratch_addr[kMaxDevices] = {};
+
+// Errors are reported by status code only: this entry point has no context
+// to hold a message.
+hsa_status static_fail(hsa_status st, const std::string&) { return st; }
+
+// Device address of the scratch array on the current device, looked up once
+// per device.  In host code the array's name is only a host-side stand-in.
+hsa_status scratch_address(void** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return static_fail(HSA_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
+  if (dev < 0 || dev >= kMaxDevices) return static_fail(HSA_ERR_INVALID_ARG, "device ordinal out of range");
+  std::lock_guard<std::mutex> lock(g_setup_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_select_scratch);
+    if (e != cudaSuccess || p == nullptr)
+      return static_fail(HSA_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    g_scratch_addr[dev] = p;
+  }
+  *out = g_scratch_addr[dev];
+  return HSA_OK;
+}
+
+bool aligned16(const void* p) { return p != nullptr && (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+hsa_status hsa_select_groups_static(const float* v_prev, const float* v_cur, int N,
+                                    const int* counts, int K, uint8_t* g, void* stream) {
+  if (N > kStaticMaxN)
+    return static_fail(HSA_ERR_SCRATCH_LIMIT,
+                       "N = " + std::to_string(N) + " is outside [1, " +
+                           std::to_string(kStaticMaxN) + "], the size of the static scratch");
+  if (N < 1) return static_fail(HSA_ERR_INVALID_ARG, "N must be >= 1");
+  if (K < 1 || K > hsa::kMaxGroups) return static_fail(HSA_ERR_INVALID_ARG, "K must be in [1, 8]");
+  if (counts == nullptr) return static_fail(HSA_ERR_INVALID_ARG, "counts is NULL");
+  long long total = 0;
+  for (int k = 0; k < K; ++k) {
+    if (counts[k] < 0) return static_fail(HSA_ERR_BUDGET, "group counts must be >= 0");
+    total += counts[k];
+  }
+  if (total != N) return static_fail(HSA_ERR_BUDGET, "group counts must sum to N");
+  if (!aligned16(v_prev) || !aligned16(v_cur) || !aligned16(g))
+    return static_fail(HSA_ERR_INVALID_ARG, "v_prev, v_cur and g must be non-NULL and 16-byte aligned");
+  void* base = nullptr;
+  if (hsa_status st = scratch_address(&base)) return st;
+  auto* bytes = static_cast<unsigned char*>(base);
+  float* score = reinterpret_cast<float*>(bytes);
+  uint32_t* cuts = reinterpret_cast<uint32_t*>(bytes + kScoreBytes);
+  int* flag = reinterpret_cast<int*>(bytes + kScoreBytes + kCutBytes);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  // the device check flag must start at zero; scores and cuts are fully rewritten
+  cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int), s);
+  if (e == cudaSuccess)
+    e = hsa::launch_select_groups_raw(s, v_prev, v_cur, N, counts, K, score, cuts, g, flag);
+  if (e != cudaSuccess) return static_fail(HSA_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
+  return HSA_OK;
+}
+
+}  // extern "C"

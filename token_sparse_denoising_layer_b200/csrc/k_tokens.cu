@@ -314,6 +314,32 @@ cudaError_t launch_select(const Ctx& c, const float* score, uint8_t* g) {
   return cudaGetLastError();
 }
 
+// Score, cut search and assignment on caller-given buffers: score [N], cuts
+// [2 * (K - 1)] words, flag [1].  Used by the allocation-free entry point.
+cudaError_t launch_select_groups_raw(cudaStream_t stream, const float* v_prev, const float* v_cur,
+                                     int N, const int* counts, int K, float* score,
+                                     uint32_t* cuts, uint8_t* g, int* flag) {
+  k_score<<<(N + 255) / 256, 256, 0, stream>>>(reinterpret_cast<const float4*>(v_prev),
+                                               reinterpret_cast<const float4*>(v_cur), score, N,
+                                               flag);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || K == 1) {
+    if (e == cudaSuccess) e = cudaMemsetAsync(g, 0, static_cast<size_t>(N), stream);
+    return e;
+  }
+  CutParams cp{};
+  int acc = 0;
+  for (int j = 0; j < K - 1; ++j) {
+    acc += counts[j];
+    cp.rank[j] = acc;
+  }
+  k_radix_cut<<<K - 1, kSelThreads, 0, stream>>>(score, N, cp, cuts, flag);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  k_assign<<<(N + 255) / 256, 256, 0, stream>>>(score, cuts, K - 1, g, N);
+  return cudaGetLastError();
+}
+
 // ============================================================ cached Euler (2.3)
 //
 // One pass over all N tokens, four channels per thread (128-bit accesses):
