@@ -6,15 +6,22 @@
 // queries against the full cached K, V (fresh rows for active tokens, stale
 // rows for skipped ones), which costs O(|A_i| * N) instead of O(N^2).
 //
-// One CTA = 128 queries x one head.  Per 128-key tile j:
-//   S_j = Q K_j^T            tcgen05.mma, fp32 in TMEM (double-buffered)
-//   P_j = exp2(S_j*c - m)    softmax warps, bf16 into 128B-swizzled smem
-//   O  += P_j V_j            tcgen05.mma, fp32 in TMEM
-// The running max m is only raised when a row's max grows by more than 2^8
-// (then O and l are rescaled in TMEM/registers); otherwise the stale max is
-// kept, which is exact because the same m scales both O and l.
-// Warp 0: TMA producer.  Warp 1: TMEM owner and MMA issuer.  Warps 2..5:
-// softmax, rescale and the output epilogue (warp w owns TMEM lanes 32*(w%4)).
+// One CTA = two 128-query tiles (t = 0, 1) of one head; both share every
+// 128-key K/V tile the producer streams in.  Per key tile j and query tile t:
+//   S_t = Q_t K_j^T          tcgen05.mma, fp32 in TMEM
+//   P_t = exp2(S_t*c - m_t)  softmax warpgroup t, written back into TMEM as
+//                            bf16 over the columns of S_t
+//   O_t += P_t V_j           tcgen05.mma with A = P_t read from TMEM
+// The two query tiles ping-pong: while warpgroup 0 turns S_0 into P_0, the
+// tensor core runs P_1 V and the next Q_1 K^T, and the other way round.
+// The running max m is raised only when a row's max grows by more than 2^8;
+// otherwise the stale max is kept, which is exact because the same m scales
+// both O and the row sum l.  A commit that signals S_t(j+1) also covers the
+// earlier P_t(j) V_j, so softmax sees a stable O_t and a free P_t region.
+//
+// Warp 0: TMA producer.  Warp 1: TMEM owner and MMA issuer.  Warps 2..5 and
+// 6..9: the softmax warpgroups of tiles 0 and 1 (warp w reads TMEM lanes
+// 32*(w%4)..+31), which also rescale O and write the output.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -31,11 +38,10 @@ namespace hsa {
 
 namespace {
 
-constexpr int kQ = 128;        // queries per CTA
+constexpr int kQ = 128;        // queries per tile
 constexpr int kKV = 128;       // keys per tile
-constexpr int kKStages = 2;
-constexpr int kVStages = 2;
-constexpr int kAttnThreads = 192;
+constexpr int kStages = 2;     // K and V ring depth
+constexpr int kAttnThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
@@ -43,21 +49,20 @@ template <int HD>
 struct AttnCfg {
   static constexpr int kRegions = HD / 64;          // 64-element (128 B) column regions
   static constexpr int kRegionBytes = 128 * 128;    // 128 rows x 128 B
-  static constexpr int kTileBytes = kRegions * kRegionBytes;  // Q, K or V tile
-  static constexpr int kPBytes = 2 * kRegionBytes;  // P: 128 x 128 bf16
-  static constexpr int kSmemData = kTileBytes * (1 + kKStages + kVStages) + kPBytes;
-  // The HD=64 kernel pads its request so that only one CTA is resident per
-  // SM: every CTA allocates all 512 TMEM columns.
+  static constexpr int kTileBytes = kRegions * kRegionBytes;  // one Q, K or V tile
+  static constexpr int kSmemData = kTileBytes * (2 + 2 * kStages);
+  // Every CTA allocates all 512 TMEM columns, so only one may be resident
+  // per SM: the HD=64 kernel pads its shared-memory request to ensure that.
   static constexpr int kSmem = (HD == 64 ? 160 * 1024 : kSmemData + 1024 + 256);
+  static constexpr uint32_t kColS0 = 0, kColS1 = 128, kColO0 = 256, kColO1 = 256 + HD;
 };
 
 struct AttnParams {
-  int n;        // active queries
-  int N;        // cached rows
-  int H;
+  int n;             // active queries
+  int N;             // cached rows
   float scale_log2;  // log2(e) / sqrt(d)
   __nv_bfloat16* o;
-  int ld;       // D
+  int ld;            // D
   int* flag;
 };
 
@@ -69,41 +74,40 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~static_cast<uintptr_t>(1023));
-  uint8_t* sQ = smem;
-  uint8_t* sK = sQ + Cfg::kTileBytes;
-  uint8_t* sV = sK + kKStages * Cfg::kTileBytes;
-  uint8_t* sP = sV + kVStages * Cfg::kTileBytes;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sP + Cfg::kPBytes);
+  uint8_t* sQ = smem;                              // [2] tiles
+  uint8_t* sK = sQ + 2 * Cfg::kTileBytes;          // [kStages]
+  uint8_t* sV = sK + kStages * Cfg::kTileBytes;    // [kStages]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(sV + kStages * Cfg::kTileBytes);
   uint64_t* q_full = bars;
-  uint64_t* k_full = bars + 1;
-  uint64_t* k_empty = k_full + kKStages;
-  uint64_t* v_full = k_empty + kKStages;
-  uint64_t* v_empty = v_full + kVStages;
-  uint64_t* s_full = v_empty + kVStages;  // [2]
-  uint64_t* p_full = s_full + 2;
-  uint64_t* pv_done = p_full + 1;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(pv_done + 1);
+  uint64_t* k_full = q_full + 1;
+  uint64_t* k_empty = k_full + kStages;
+  uint64_t* v_full = k_empty + kStages;
+  uint64_t* v_empty = v_full + kStages;
+  uint64_t* s_full = v_empty + kStages;  // [2] per query tile
+  uint64_t* p_full = s_full + 2;         // [2]
+  uint64_t* o_done = p_full + 2;         // [2]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * kQ;
+  const int q0 = blockIdx.x * (2 * kQ);
   const int h = blockIdx.y;
   const int col0 = h * HD;
   const int nkv = (p.N + kKV - 1) / kKV;
+  const int ntile = (q0 + kQ < p.n) ? 2 : 1;  // second query tile empty on the last CTA
 
   if (threadIdx.x == 0) {
     mbar_init(q_full, 1);
-    for (int s = 0; s < kKStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&k_full[s], 1);
       mbar_init(&k_empty[s], 1);
-    }
-    for (int s = 0; s < kVStages; ++s) {
       mbar_init(&v_full[s], 1);
       mbar_init(&v_empty[s], 1);
     }
-    mbar_init(&s_full[0], 1);
-    mbar_init(&s_full[1], 1);
-    mbar_init(p_full, 128);
-    mbar_init(pv_done, 1);
+    for (int t = 0; t < 2; ++t) {
+      mbar_init(&s_full[t], 1);
+      mbar_init(&p_full[t], 4);  // one arrival per softmax warp
+      mbar_init(&o_done[t], 1);
+    }
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -119,35 +123,35 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem;              // S buffers at columns 0 and 128
-  const uint32_t tO = tmem + 2 * kKV;    // O at column 256
   bool ok = true;
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const uint64_t keep = l2_policy_evict_last();  // K/V of a head is shared by its q-tiles
-      mbar_arrive_expect_tx(q_full, Cfg::kTileBytes);
-      for (int r = 0; r < Cfg::kRegions; ++r)
-        tma_load_2d(sQ + r * Cfg::kRegionBytes, &tmQ, q_full, col0 + 64 * r, q0);
-      for (int j = 0; j < nkv && ok; ++j) {
-        const int ks = j % kKStages;
-        if (!mbar_wait(&k_empty[ks], ((j / kKStages) & 1) ^ 1)) {
+      const uint64_t keep = l2_policy_evict_last();  // a head's K/V is shared by its q-tiles
+      mbar_arrive_expect_tx(q_full, ntile * Cfg::kTileBytes);
+      for (int t = 0; t < ntile; ++t)
+        for (int r = 0; r < Cfg::kRegions; ++r)
+          tma_load_2d(sQ + t * Cfg::kTileBytes + r * Cfg::kRegionBytes, &tmQ, q_full,
+                      col0 + 64 * r, q0 + t * kQ);
+      for (int j = 0; j < nkv; ++j) {
+        const int s = j % kStages;
+        const uint32_t ph = ((j / kStages) & 1) ^ 1;
+        if (!mbar_wait(&k_empty[s], ph)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&k_full[ks], Cfg::kTileBytes);
+        mbar_arrive_expect_tx(&k_full[s], Cfg::kTileBytes);
         for (int r = 0; r < Cfg::kRegions; ++r)
-          tma_load_2d_hint(sK + ks * Cfg::kTileBytes + r * Cfg::kRegionBytes, &tmK, &k_full[ks],
+          tma_load_2d_hint(sK + s * Cfg::kTileBytes + r * Cfg::kRegionBytes, &tmK, &k_full[s],
                            col0 + 64 * r, j * kKV, keep);
-        const int vs = j % kVStages;
-        if (!mbar_wait(&v_empty[vs], ((j / kVStages) & 1) ^ 1)) {
+        if (!mbar_wait(&v_empty[s], ph)) {
           ok = false;
           break;
         }
-        mbar_arrive_expect_tx(&v_full[vs], Cfg::kTileBytes);
+        mbar_arrive_expect_tx(&v_full[s], Cfg::kTileBytes);
         for (int r = 0; r < Cfg::kRegions; ++r)
-          tma_load_2d_hint(sV + vs * Cfg::kTileBytes + r * Cfg::kRegionBytes, &tmV, &v_full[vs],
+          tma_load_2d_hint(sV + s * Cfg::kTileBytes + r * Cfg::kRegionBytes, &tmV, &v_full[s],
                            col0 + 64 * r, j * kKV, keep);
       }
     }
@@ -156,145 +160,159 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     if (lane == 0) {
       constexpr uint32_t idS = idesc_bf16(kQ, kKV, false, false);
       constexpr uint32_t idPV = idesc_bf16(kQ, HD, false, true);
-      const uint32_t q_addr = smem_u32(sQ);
-      const uint32_t p_addr = smem_u32(sP);
-      auto issue_s = [&](int j) -> bool {
-        const int ks = j % kKStages;
-        if (!mbar_wait(&k_full[ks], (j / kKStages) & 1)) return false;
-        tc_fence_after();
-        const uint32_t k_addr = smem_u32(sK + ks * Cfg::kTileBytes);
+      // S_t = Q_t K^T for the K tile in stage s
+      auto issue_s = [&](int t, int s) {
+        const uint32_t q_addr = smem_u32(sQ + t * Cfg::kTileBytes);
+        const uint32_t k_addr = smem_u32(sK + s * Cfg::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * Cfg::kRegionBytes + (kk & 3) * 32;
-          umma_bf16(tS + (j & 1) * kKV, sdesc_sw128(q_addr + off, 16, 1024),
+          umma_bf16(tmem + (t == 0 ? Cfg::kColS0 : Cfg::kColS1), sdesc_sw128(q_addr + off, 16, 1024),
                     sdesc_sw128(k_addr + off, 16, 1024), idS, kk > 0 ? 1u : 0u);
         }
-        umma_commit(&s_full[j & 1]);
-        umma_commit(&k_empty[ks]);
-        return true;
       };
-      if (!mbar_wait(q_full, 0)) ok = false;
-      if (ok && !issue_s(0)) ok = false;
-      for (int j = 0; j < nkv && ok; ++j) {
-        if (j + 1 < nkv && !issue_s(j + 1)) {
-          ok = false;
-          break;
-        }
-        if (!mbar_wait(p_full, j & 1)) {
-          ok = false;
-          break;
-        }
-        const int vs = j % kVStages;
-        if (!mbar_wait(&v_full[vs], (j / kVStages) & 1)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t v_addr = smem_u32(sV + vs * Cfg::kTileBytes);
+      // O_t (+)= P_t V for the V tile in stage s; P_t sits in the S_t columns
+      auto issue_pv = [&](int t, int s, bool acc) {
+        const uint32_t v_addr = smem_u32(sV + s * Cfg::kTileBytes);
 #pragma unroll
         for (int kk = 0; kk < kKV / 16; ++kk) {
-          const uint32_t a_off = (kk >> 2) * Cfg::kRegionBytes + (kk & 3) * 32;
-          // V tile is MN-major for this product: rows = keys (K), 128 B of head dim
-          // per row; 16 keys per step = 2048 B; regions of 64 dims are LBO apart.
-          umma_bf16(tO, sdesc_sw128(p_addr + a_off, 16, 1024),
-                    sdesc_sw128(v_addr + kk * 2048, Cfg::kRegionBytes, 1024), idPV,
-                    (j > 0 || kk > 0) ? 1u : 0u);
+          // V is MN-major here: rows = keys (K), 128 B of head dim per row,
+          // 16 keys per step = 2048 B, 64-dim regions are LBO apart.
+          umma_bf16_ta(tmem + (t == 0 ? Cfg::kColO0 : Cfg::kColO1),
+                       tmem + (t == 0 ? Cfg::kColS0 : Cfg::kColS1) + kk * 8,
+                       sdesc_sw128(v_addr + kk * 2048, Cfg::kRegionBytes, 1024), idPV,
+                       (acc || kk > 0) ? 1u : 0u);
         }
-        umma_commit(pv_done);
-        umma_commit(&v_empty[vs]);
+      };
+      ok = mbar_wait(q_full, 0) && mbar_wait(&k_full[0], 0);
+      if (ok) {
+        tc_fence_after();
+        for (int t = 0; t < ntile; ++t) {
+          issue_s(t, 0);
+          umma_commit(&s_full[t]);
+        }
+        umma_commit(&k_empty[0]);
+      }
+      for (int j = 0; j < nkv && ok; ++j) {
+        const int s = j % kStages;
+        const int s1 = (j + 1) % kStages;
+        for (int t = 0; t < ntile && ok; ++t) {
+          if (!mbar_wait(&p_full[t], j & 1)) {
+            ok = false;
+            break;
+          }
+          if (t == 0 && !mbar_wait(&v_full[s], (j / kStages) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          issue_pv(t, s, j > 0);
+          if (t == ntile - 1) umma_commit(&v_empty[s]);
+          if (j + 1 < nkv) {
+            if (t == 0 && !mbar_wait(&k_full[s1], ((j + 1) / kStages) & 1)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            issue_s(t, s1);
+            umma_commit(&s_full[t]);
+            if (t == ntile - 1) umma_commit(&k_empty[s1]);
+          } else {
+            umma_commit(&o_done[t]);
+          }
+        }
       }
     }
   } else {
-    // ------------------------------------------------------------ softmax warps
-    const int qd = warp & 3;
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = (warp - 2) >> 2;  // query tile of this warpgroup
+    const int qd = warp & 3;        // TMEM lane quarter
     const int row = 32 * qd + lane;
     const uint32_t lane_base = static_cast<uint32_t>(32 * qd) << 16;
+    const uint32_t tS = tmem + lane_base + (t == 0 ? Cfg::kColS0 : Cfg::kColS1);
+    const uint32_t tO = tmem + lane_base + (t == 0 ? Cfg::kColO0 : Cfg::kColO1);
+    const bool active = t < ntile;
     float m_run = -INFINITY, l_run = 0.f;
-    uint8_t* prow = sP + row * 128;
-    const int sw = row & 7;
-    for (int j = 0; j < nkv; ++j) {
-      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[j & 1], (j >> 1) & 1))) {
+    for (int j = 0; j < nkv && active; ++j) {
+      if (!__all_sync(0xffffffffu, mbar_wait(&s_full[t], j & 1))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float s[kKV];
+      const int valid = p.N - j * kKV;  // keys past N are zero-filled: mask them
+      // pass 1: row max of this tile
+      float tmax = -INFINITY;
 #pragma unroll
       for (int c = 0; c < kKV / 32; ++c) {
         uint32_t r[32];
-        tmem_ld32(tS + lane_base + (j & 1) * kKV + 32 * c, r);
+        tmem_ld32(tS + 32 * c, r);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s[32 * c + e] = __uint_as_float(r[e]);
+        for (int e = 0; e < 32; ++e)
+          if (32 * c + e < valid) tmax = fmaxf(tmax, __uint_as_float(r[e]));
       }
-      const int valid = p.N - j * kKV;  // keys past N are zero-filled: mask them
-      float tmax = -INFINITY;
-#pragma unroll
-      for (int e = 0; e < kKV; ++e) {
-        s[e] = (e < valid) ? s[e] * p.scale_log2 : -INFINITY;
-        tmax = fmaxf(tmax, s[e]);
-      }
+      tmax *= p.scale_log2;
       const bool raise = tmax > m_run + kRescaleThreshold;
       const float m_use = raise ? tmax : m_run;
       const float alpha = raise ? ex2_approx(m_run - m_use) : 1.0f;
-      // PV_{j-1} must be done before P is overwritten and before O is rescaled.
-      if (j > 0 && !__all_sync(0xffffffffu, mbar_wait(pv_done, (j - 1) & 1))) {
-        ok = false;
-        break;
-      }
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < kKV / 8; ++c) {  // 16-byte chunks of 8 keys
-        float pv[8];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          pv[e] = ex2_approx(s[8 * c + e] - m_use);
-          rs += pv[e];
-        }
-        const uint4 w = make_uint4(pack_bf16(pv[0], pv[1]), pack_bf16(pv[2], pv[3]),
-                                   pack_bf16(pv[4], pv[5]), pack_bf16(pv[6], pv[7]));
-        const int region = c >> 3, cc = c & 7;
-        *reinterpret_cast<uint4*>(prow + region * Cfg::kRegionBytes + ((cc ^ sw) << 4)) = w;
-      }
-      l_run = l_run * alpha + rs;
-      m_run = m_use;
+      // O_t is stable here: the commit behind s_full covers P_t(j-1) V_{j-1}.
       if (j > 0 && __any_sync(0xffffffffu, raise)) {
 #pragma unroll 1
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t r[32];
-          tmem_ld32(tO + lane_base + 32 * c, r);
+          tmem_ld32(tO + 32 * c, r);
 #pragma unroll
           for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-          tmem_st32(tO + lane_base + 32 * c, r);
+          tmem_st32(tO + 32 * c, r);
         }
       }
-      fence_proxy_async_smem();
+      // pass 2: P = exp2(S*c - m) as bf16 pairs, then into the S_t columns
+      uint32_t w[kKV / 2];
+      float rs = 0.f;
+#pragma unroll
+      for (int c = 0; c < kKV / 32; ++c) {
+        uint32_t r[32];
+        tmem_ld32(tS + 32 * c, r);
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float a = (32 * c + e < valid) ? ex2_approx(fmaf(__uint_as_float(r[e]), p.scale_log2, -m_use)) : 0.f;
+          float b = (32 * c + e + 1 < valid) ? ex2_approx(fmaf(__uint_as_float(r[e + 1]), p.scale_log2, -m_use)) : 0.f;
+          rs += a + b;
+          w[16 * c + e / 2] = pack_bf16(a, b);
+        }
+      }
+      tmem_st64(tS, w);
+      l_run = l_run * alpha + rs;
+      m_run = m_use;
       tc_fence_before();
-      mbar_arrive(p_full);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&p_full[t]);
     }
     // epilogue: O / l -> bf16 rows of the compact output
-    if (ok && __all_sync(0xffffffffu, mbar_wait(pv_done, (nkv - 1) & 1))) {
-      tc_fence_after();
-      const float inv = 1.0f / l_run;
-      const int qrow = q0 + row;
-      __nv_bfloat16* orow = p.o + static_cast<size_t>(qrow) * p.ld + col0;
+    if (active && ok) {
+      if (__all_sync(0xffffffffu, mbar_wait(&o_done[t], 0))) {
+        tc_fence_after();
+        const float inv = 1.0f / l_run;
+        const int qrow = q0 + t * kQ + row;
+        __nv_bfloat16* orow = p.o + static_cast<size_t>(qrow) * p.ld + col0;
 #pragma unroll 1
-      for (int c = 0; c < HD / 32; ++c) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld32(tO + lane_base + 32 * c, r);
-        if (qrow < p.n) {
-          uint4* d4 = reinterpret_cast<uint4*>(orow + 32 * c);
+        for (int c = 0; c < HD / 32; ++c) {
+          uint32_t r[32];
+          __syncwarp();
+          tmem_ld32(tO + 32 * c, r);
+          if (qrow < p.n) {
+            uint4* d4 = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
-          for (int v = 0; v < 4; ++v)
-            d4[v] = make_uint4(
-                pack_bf16(__uint_as_float(r[8 * v]) * inv, __uint_as_float(r[8 * v + 1]) * inv),
-                pack_bf16(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv),
-                pack_bf16(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv),
-                pack_bf16(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv));
+            for (int v = 0; v < 4; ++v)
+              d4[v] = make_uint4(
+                  pack_bf16(__uint_as_float(r[8 * v]) * inv, __uint_as_float(r[8 * v + 1]) * inv),
+                  pack_bf16(__uint_as_float(r[8 * v + 2]) * inv, __uint_as_float(r[8 * v + 3]) * inv),
+                  pack_bf16(__uint_as_float(r[8 * v + 4]) * inv, __uint_as_float(r[8 * v + 5]) * inv),
+                  pack_bf16(__uint_as_float(r[8 * v + 6]) * inv, __uint_as_float(r[8 * v + 7]) * inv));
+          }
         }
+      } else {
+        ok = false;
       }
-    } else {
-      ok = false;
     }
   }
   if (!ok) atomicOr(p.flag, DEV_TIMEOUT);
@@ -317,7 +335,6 @@ cudaError_t launch_hd(const Ctx& c, const void* q, int n, const void* kc, const 
   AttnParams p{};
   p.n = n;
   p.N = N;
-  p.H = c.cfg.H;
   p.scale_log2 = static_cast<float>(1.4426950408889634 / sqrt(static_cast<double>(HD)));
   p.o = static_cast<__nv_bfloat16*>(o);
   p.ld = D;
@@ -330,7 +347,7 @@ cudaError_t launch_hd(const Ctx& c, const void* q, int n, const void* kc, const 
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const dim3 grid((n + kQ - 1) / kQ, c.cfg.H);
+  const dim3 grid((n + 2 * kQ - 1) / (2 * kQ), c.cfg.H);
   k_attn<HD><<<grid, kAttnThreads, smem, c.stream>>>(tq, tk, tv, p);
   return cudaGetLastError();
 }
