@@ -80,3 +80,4 @@ def test_binding_fails_loudly_without_library(monkeypatch):
     monkeypatch.setattr(abi, "LIB_PATH", "/nonexistent/libhsa.so")
     with pytest.raises(RuntimeError, match="missing"):
         abi.load()
+

@@ -8,9 +8,12 @@
 // section 2.2): fresh K/V rows are scattered into the KV cache rows idx[m],
 // and out-projection / MLP results are added into residual rows idx[m].
 //
-// CTA tile 128 x BN (BN = 256 or 128), K-block 64, a multi-stage TMA ring.
-// Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs (one thread),
-// warps 2..5 drain TMEM and run the epilogue.
+// Persistent: one CTA per SM walks its share of the 128 x BN output tiles
+// (BN = 256 or 128), K-block 64, through a multi-stage TMA ring that runs on
+// across tiles.  Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs (one
+// thread) into one of two TMEM accumulators, warps 2..5 drain the other
+// accumulator and run the epilogue, so a tile's epilogue overlaps the next
+// tile's main loop.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -95,7 +98,7 @@ __device__ __forceinline__ void add_f32x32(float* dst, const uint32_t (&r)[32]) 
 template <int BN>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     k_gemm(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-           EpiParams p) {
+           EpiParams p, int n_tiles, int total_tiles) {
   using Cfg = GemmCfg<BN>;
   constexpr int S = Cfg::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -105,11 +108,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint8_t* sB = smem + S * Cfg::kABytes;
   uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * Cfg::kBBytes);
   uint64_t* empty = full + S;
-  uint64_t* accf = empty + S;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(accf + 1);
+  uint64_t* acc_full = empty + S;     // [2] accumulator buffer ready for the epilogue
+  uint64_t* acc_empty = acc_full + 2; // [2] accumulator buffer drained
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int n0 = blockIdx.x * BN, m0 = blockIdx.y * kBM;
   const int nk = p.Kd / kBK;
 
   if (threadIdx.x == 0) {
@@ -117,7 +120,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    mbar_init(accf, 1);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+    }
     fence_barrier_init();
   }
   if (warp == 0 && lane == 0) {
@@ -125,7 +131,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, BN);
+    tmem_alloc(tmem_slot, 2 * BN);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -134,66 +140,81 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t tmem = *tmem_slot;
   bool ok = true;
 
+  // Tiles are visited t = blockIdx.x, +gridDim.x, ...; tile t covers rows
+  // (t / n_tiles) * 128 and columns (t % n_tiles) * BN, so tiles running at the
+  // same time share A row blocks and sweep the (L2-resident) weight.
   if (warp == 0) {
     if (lane == 0) {
-      int issued = 0;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (!mbar_wait(&empty[s], ph ^ 1)) {
-          ok = false;
-          break;
+      int it = 0;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x) {
+        const int m0 = (t / n_tiles) * kBM, n0 = (t % n_tiles) * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
+          tma_load_2d(sA + s * Cfg::kABytes, &tmA, &full[s], kb * kBK, m0);
+          tma_load_2d(sB + s * Cfg::kBBytes, &tmB, &full[s], kb * kBK, n0);
         }
-        mbar_arrive_expect_tx(&full[s], Cfg::kStageBytes);
-        tma_load_2d(sA + s * Cfg::kABytes, &tmA, &full[s], kb * kBK, m0);
-        tma_load_2d(sB + s * Cfg::kBBytes, &tmB, &full[s], kb * kBK, n0);
-        issued = kb + 1;
       }
       if (!ok) {  // let copies already in flight land before the CTA exits
-        for (int kb = issued > S ? issued - S : 0; kb < issued; ++kb)
-          (void)mbar_wait(&full[kb % S], (kb / S) & 1);
+        for (int k = it > S ? it - S : 0; k < it; ++k) (void)mbar_wait(&full[k % S], (k / S) & 1);
       }
     }
   } else if (warp == 1) {
     if (lane == 0) {
       constexpr uint32_t idesc = idesc_bf16(kBM, BN, false, false);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (!mbar_wait(&full[s], ph)) {
+      int it = 0, lt = 0;
+      for (int t = blockIdx.x; t < total_tiles && ok; t += gridDim.x, ++lt) {
+        const int b = lt & 1;
+        if (!mbar_wait(&acc_empty[b], ((lt >> 1) & 1) ^ 1)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t a0 = smem_u32(sA + s * Cfg::kABytes);
-        const uint32_t b0 = smem_u32(sB + s * Cfg::kBBytes);
+        const uint32_t acc = tmem + b * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(&full[s], (it / S) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * Cfg::kABytes);
+          const uint32_t b0 = smem_u32(sB + s * Cfg::kBBytes);
 #pragma unroll
-        for (int kk = 0; kk < kBK / 16; ++kk) {
-          const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
-          const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
-          umma_bf16(tmem, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kBK / 16; ++kk) {
+            const uint64_t ad = sdesc_sw128(a0 + kk * 32, 16, 1024);
+            const uint64_t bd = sdesc_sw128(b0 + kk * 32, 16, 1024);
+            umma_bf16(acc, ad, bd, idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[s]);
         }
-        umma_commit(&empty[s]);
+        umma_commit(&acc_full[b]);
       }
-      umma_commit(accf);
     }
   } else {
     // epilogue: warp w reads TMEM lanes [32*(w%4), +32) = tile rows
     const int q = warp & 3;
     const int row = 32 * q + lane;
-    const int m = m0 + row;
-    const bool waited = __all_sync(0xffffffffu, mbar_wait(accf, 0));
-    if (!waited) {
-      ok = false;
-    } else {
+    int lt = 0;
+    for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++lt) {
+      const int b = lt & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[b], (lt >> 1) & 1))) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
+      const int m = (t / n_tiles) * kBM + row, n0 = (t % n_tiles) * BN;
       const bool mrow = m < p.M;
       int32_t dst_row = 0;
       if (mrow && (p.epi == EPI_QKV || p.epi == EPI_RESID)) {
         dst_row = __ldg(p.idx + m);
         if (!row_ok(dst_row, p.N, p.flag)) dst_row = -1;
       }
-      const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16);
+      const uint32_t tbase = tmem + b * BN + (static_cast<uint32_t>(32 * q) << 16);
 #pragma unroll 1
       for (int c0 = 0; c0 < BN; c0 += 32) {
         uint32_t r[32];
@@ -226,6 +247,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
         }
       }
+      // the buffer may be refilled once every lane's TMEM reads are done
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[b]);
     }
   }
   if (!ok) atomicOr(p.flag, DEV_TIMEOUT);
@@ -233,7 +258,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, BN);
+    tmem_dealloc(tmem, 2 * BN);
   }
 }
 
@@ -263,8 +288,10 @@ cudaError_t launch_bn(const Ctx& c, const GemmArgs& a, std::string* why) {
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const dim3 grid((a.Ncols + BN - 1) / BN, (a.M + kBM - 1) / kBM);
-  k_gemm<BN><<<grid, kGemmThreads, smem, c.stream>>>(ta, tb, p);
+  const int n_tiles = (a.Ncols + BN - 1) / BN;
+  const int total = n_tiles * ((a.M + kBM - 1) / kBM);
+  const int grid = total < c.num_sms ? total : c.num_sms;
+  k_gemm<BN><<<grid, kGemmThreads, smem, c.stream>>>(ta, tb, p, n_tiles, total);
   return cudaGetLastError();
 }
 
