@@ -240,16 +240,21 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       tc_fence_after();
       const int valid = p.N - j * kKV;  // keys past N are zero-filled: mask them
-      // pass 1: row max of this tile
-      float tmax = -INFINITY;
+      // the whole S row of this tile in one TMEM load
+      uint32_t sr[kKV];
+      tmem_ld128(tS, sr);
+      if (valid < kKV) {
 #pragma unroll
-      for (int c = 0; c < kKV / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + 32 * c, r);
-#pragma unroll
-        for (int e = 0; e < 32; ++e)
-          if (32 * c + e < valid) tmax = fmaxf(tmax, __uint_as_float(r[e]));
+        for (int e = 0; e < kKV; ++e)
+          if (e >= valid) sr[e] = __float_as_uint(-INFINITY);
       }
+      float mx[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mx[u] = __uint_as_float(sr[u]);
+#pragma unroll
+      for (int e = 8; e < kKV; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sr[e]));
+      float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
       tmax *= p.scale_log2;
       const bool raise = tmax > m_run + kRescaleThreshold;
       const float m_use = raise ? tmax : m_run;
@@ -265,21 +270,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           tmem_st32(tO + 32 * c, r);
         }
       }
-      // pass 2: P = exp2(S*c - m) as bf16 pairs, then into the S_t columns
+      // P = exp2(S*c - m) as bf16 pairs, written over the S_t columns
       uint32_t w[kKV / 2];
-      float rs = 0.f;
+      float rsum[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int c = 0; c < kKV / 32; ++c) {
-        uint32_t r[32];
-        tmem_ld32(tS + 32 * c, r);
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float a = (32 * c + e < valid) ? ex2_approx(fmaf(__uint_as_float(r[e]), p.scale_log2, -m_use)) : 0.f;
-          float b = (32 * c + e + 1 < valid) ? ex2_approx(fmaf(__uint_as_float(r[e + 1]), p.scale_log2, -m_use)) : 0.f;
-          rs += a + b;
-          w[16 * c + e / 2] = pack_bf16(a, b);
-        }
+      for (int e = 0; e < kKV; e += 2) {
+        const float a = ex2_approx(fmaf(__uint_as_float(sr[e]), p.scale_log2, -m_use));
+        const float b = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), p.scale_log2, -m_use));
+        rsum[(e >> 1) & 3] += a + b;
+        w[e / 2] = pack_bf16(a, b);
       }
+      const float rs = (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
       tmem_st64(tS, w);
       l_run = l_run * alpha + rs;
       m_run = m_use;
