@@ -271,16 +271,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
       }
       // P = exp2(S*c - m) as bf16 pairs, written over the S_t columns
+      // (packed f32x2 arithmetic: two lanes per FMA/add instruction)
       uint32_t w[kKV / 2];
-      float rsum[4] = {0.f, 0.f, 0.f, 0.f};
+      float rs0[4] = {0.f, 0.f, 0.f, 0.f}, rs1[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int e = 0; e < kKV; e += 2) {
-        const float a = ex2_approx(fmaf(__uint_as_float(sr[e]), p.scale_log2, -m_use));
-        const float b = ex2_approx(fmaf(__uint_as_float(sr[e + 1]), p.scale_log2, -m_use));
-        rsum[(e >> 1) & 3] += a + b;
+        float xa, xb;
+        fma2(xa, xb, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), p.scale_log2, -m_use);
+        const float a = ex2_approx(xa);
+        const float b = ex2_approx(xb);
+        add2(rs0[(e >> 1) & 3], rs1[(e >> 1) & 3], a, b);
         w[e / 2] = pack_bf16(a, b);
       }
-      const float rs = (rsum[0] + rsum[1]) + (rsum[2] + rsum[3]);
+      const float rs = ((rs0[0] + rs1[0]) + (rs0[1] + rs1[1])) + ((rs0[2] + rs1[2]) + (rs0[3] + rs1[3]));
       tmem_st64(tS, w);
       l_run = l_run * alpha + rs;
       m_run = m_use;

@@ -35,7 +35,9 @@ constexpr int kGemmThreads = 192;
 
 template <int BN>
 struct GemmCfg {
-  static constexpr int kStages = BN == 256 ? 4 : 6;
+  static constexpr int kStages = BN == 256 ? 4 : BN == 192 ? 5 : 6;
+  // two accumulators of BN fp32 columns, allocated as a power of two
+  static constexpr uint32_t kTmemCols = 2 * BN <= 256 ? 256 : 512;
   static constexpr int kABytes = kBM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
@@ -131,7 +133,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     tma_prefetch_desc(&tmB);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_slot, 2 * BN);
+    tmem_alloc(tmem_slot, Cfg::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -258,7 +260,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 2 * BN);
+    tmem_dealloc(tmem, Cfg::kTmemCols);
   }
 }
 
@@ -303,7 +305,21 @@ cudaError_t launch_gemm(const Ctx& c, const GemmArgs& a, std::string* why) {
     if (why) *why = "GEMM needs K % 64 == 0 and Ncols % 32 == 0";
     return cudaErrorInvalidValue;
   }
-  if (a.Ncols % 256 == 0) return launch_bn<256>(c, a, why);
+  // Pick the tile width with the fewest tile-waves x tile width, where a
+  // narrower tile costs a little more per column (more smem traffic per FLOP).
+  const int mt = (a.M + kBM - 1) / kBM;
+  auto cost = [&](int bn, double per_col) {
+    const long tiles = static_cast<long>(mt) * ((a.Ncols + bn - 1) / bn);
+    const long waves = (tiles + c.num_sms - 1) / c.num_sms;
+    return static_cast<double>(waves) * bn * per_col;
+  };
+  double best = 1e300;
+  int bn = 128;
+  if (a.Ncols % 256 == 0 && cost(256, 1.0) < best) best = cost(256, 1.0), bn = 256;
+  if (a.Ncols % 192 == 0 && cost(192, 1.03) < best) best = cost(192, 1.03), bn = 192;
+  if (cost(128, 1.12) < best) best = cost(128, 1.12), bn = 128;
+  if (bn == 256) return launch_bn<256>(c, a, why);
+  if (bn == 192) return launch_bn<192>(c, a, why);
   return launch_bn<128>(c, a, why);
 }
 
