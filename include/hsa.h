@@ -118,6 +118,15 @@ hsa_status hsa_set_stream(hsa_ctx* ctx, void* stream);
 hsa_status hsa_sync_check(hsa_ctx* ctx);
 
 /*
+ * Failure-detection self-test.  Launches one kernel whose mbarrier wait is
+ * never satisfied; the same bounded wait the pipelined kernels use gives up
+ * after timeout_us microseconds (1..2000000) and records a timeout in the
+ * device flag.  The next hsa_sync_check then returns HSA_ERR_TIMEOUT and
+ * clears the flag; the context stays usable.  Nothing faults or hangs.
+ */
+hsa_status hsa_selftest_timeout(hsa_ctx* ctx, int timeout_us);
+
+/*
  * |A_i| computed on the host from the group counts ([TS] 2.1): the sum of n_k
  * over the groups active at iteration i.  Valid when g holds exactly counts[k]
  * tokens of group k, which the initial split and hsa_select_groups guarantee.

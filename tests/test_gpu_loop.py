@@ -18,7 +18,7 @@ from token_sparse_denoising_layer_b200.loop import HsaLoop, sigma_schedule
 pytestmark = pytest.mark.gpu
 
 
-def _setup(budgets=(8, 4), fractions=(0.5, 0.5)):
+def _setup(budgets=(8, 4), fractions=(0.5, 0.5), m=0):
     spec = synth.WORKLOADS["tiny_dit"]
     sh = spec["shape"]
     T = spec["T"]
@@ -26,7 +26,7 @@ def _setup(budgets=(8, 4), fractions=(0.5, 0.5)):
     w = synth.model_weights(sh, spec["seed"])
     layers = [tuple(bf(lw[k]) for k in ("w_qkv", "w_o", "w_1", "w_2")) for lw in w["layers"]]
     loop = HsaLoop(sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]), T,
-                   list(budgets), counts, shift=spec["shift"])
+                   list(budgets), counts, shift=spec["shift"], m=m)
     x0 = synth.latent(sh.N, 16, spec["seed"])
     g0 = synth.random_split(sh.N, counts, spec["seed"])
     return sh, T, counts, w, loop, x0, g0
@@ -81,3 +81,20 @@ def test_loop_is_deterministic():
         kc.zero_()
     loop.run()
     assert (host(loop.x) == a).all()
+
+
+def test_phase_window_loop_drift():
+    """Phase-aware window (first and last m iterations run all tokens) through
+    the whole loop, against the oracle with the same window."""
+    need_gpu()
+    sh, T, counts, w, loop, x0, g0 = _setup(budgets=(8, 4, 2), fractions=(0.4, 0.3, 0.3), m=2)
+    assert [loop.n_active(i) for i in range(T)] == [
+        O.n_active(i, T, [8, 4, 2], counts, 2) for i in range(T)]
+    assert loop.n_active(0) == loop.n_active(7) == sh.N
+    loop.reset(x0, g0)
+    loop.run(regroup=False)
+    xr = O.run_loop(w, x0, g0, T, [8, 4, 2], counts, O.sigma_schedule(T, 1.0), sh.H, m=2,
+                    regroup=False)
+    d = _drift(host(loop.x), xr)
+    print(f"tiny DiT with phase window m=2: x_T drift {d:.3e}")
+    assert d <= 2e-2

@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(PKG, "libhsa.so")
 # Every symbol the header declares, in header order.
 SYMBOLS = [
     "hsa_create", "hsa_destroy", "hsa_last_error", "hsa_set_stream", "hsa_sync_check",
-    "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
+    "hsa_selftest_timeout", "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
     "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_linear", "hsa_kv_scatter",
     "hsa_attention", "hsa_out_proj_residual", "hsa_mlp_residual", "hsa_layer_forward",
     "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_step", "hsa_select_groups_static",
@@ -81,6 +81,7 @@ def load() -> ctypes.CDLL:
         "hsa_last_error": (ctypes.c_char_p, [P]),
         "hsa_set_stream": (I, [P, P]),
         "hsa_sync_check": (I, [P]),
+        "hsa_selftest_timeout": (I, [P, I]),
         "hsa_n_active": (I, [P, I]),
         "hsa_schedule": (I, [P, I, P, P, P, P, ctypes.POINTER(I)]),
         "hsa_score": (I, [P, P, P, P]),
@@ -174,6 +175,10 @@ def hsa_set_stream(ctx: Context, stream) -> None:
 
 def hsa_sync_check(ctx: Context) -> None:
     _check(ctx.ptr, load().hsa_sync_check(ctx.ptr))
+
+
+def hsa_selftest_timeout(ctx: Context, timeout_us: int) -> None:
+    _check(ctx.ptr, load().hsa_selftest_timeout(ctx.ptr, timeout_us))
 
 
 def hsa_n_active(ctx: Context, i: int) -> int:

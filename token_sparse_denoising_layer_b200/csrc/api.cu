@@ -211,6 +211,14 @@ hsa_status hsa_sync_check(hsa_ctx* ctx) {
   return fail(ctx, (flag & hsa::DEV_TIMEOUT) ? HSA_ERR_TIMEOUT : HSA_ERR_DEVICE_CHECK, msg);
 }
 
+hsa_status hsa_selftest_timeout(hsa_ctx* ctx, int timeout_us) {
+  HSA_CHECK_CTX(ctx);
+  if (timeout_us < 1 || timeout_us > 2000000)
+    return fail(ctx, HSA_ERR_INVALID_ARG, "timeout_us must be in [1, 2000000]");
+  return launched(ctx, hsa::launch_selftest_timeout(ctx->c, 1000ull * timeout_us),
+                  "selftest_timeout");
+}
+
 int hsa_n_active(const hsa_ctx* ctx, int i) {
   if (ctx == nullptr || i < 0 || i >= ctx->c.T) return -1;
   const Ctx& x = ctx->c;

@@ -52,6 +52,7 @@ cudaError_t launch_select(const Ctx& c, const float* score, uint8_t* g);
 cudaError_t launch_select_groups_raw(cudaStream_t stream, const float* v_prev, const float* v_cur,
                                      int N, const int* counts, int K, float* score,
                                      uint32_t* cuts, uint8_t* g, int* flag);
+cudaError_t launch_selftest_timeout(const Ctx& c, uint64_t limit_ns);
 cudaError_t launch_euler(const Ctx& c, float* x, float* v_hat, float* v_hat_prev,
                          const float* v_fresh, const uint8_t* mask, float s0, float s1);
 cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, int n, void* u);

@@ -340,6 +340,24 @@ cudaError_t launch_select_groups_raw(cudaStream_t stream, const float* v_prev, c
   return cudaGetLastError();
 }
 
+// ============================================================ failure-detection self-test
+//
+// One thread waits on an mbarrier that nothing ever arrives at, through the
+// same bounded wait the pipelined kernels use.  The wait gives up after
+// limit_ns, the kernel records DEV_TIMEOUT and returns: no trap, no hang.
+
+__global__ void k_selftest_timeout(uint64_t limit_ns, int* flag) {
+  __shared__ uint64_t bar;
+  mbar_init(&bar, 1);
+  fence_barrier_init();
+  if (!mbar_wait(&bar, 0, limit_ns)) atomicOr(flag, DEV_TIMEOUT);
+}
+
+cudaError_t launch_selftest_timeout(const Ctx& c, uint64_t limit_ns) {
+  k_selftest_timeout<<<1, 1, 0, c.stream>>>(limit_ns, c.flag);
+  return cudaGetLastError();
+}
+
 // ============================================================ cached Euler (2.3)
 //
 // One pass over all N tokens, four channels per thread (128-bit accesses):
