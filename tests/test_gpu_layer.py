@@ -60,6 +60,8 @@ def test_ln_gather(N, D, a):
     (1000, 128, 2, 1000, 1.0),    # head_dim 64
     (130, 128, 1, 1, 8.0),        # one query, key tail of 2
     (4096, 1536, 12, 200, 3.0),
+    (12800, 256, 2, 12800, 2.0),  # 100 work units: no key-range split
+    (2000, 128, 1, 1999, 3.0),    # 8 units split 18 ways, ragged last tile
 ])
 def test_attention(N, D, H, n, q_scale):
     need_gpu()

@@ -162,6 +162,12 @@ hsa_status hsa_create(const hsa_model_cfg* cfg, int T, const int* budgets, const
   if (e == cudaSuccess) e = cudaMalloc(&x.q, nd);
   if (e == cudaSuccess) e = cudaMalloc(&x.o, nd);
   if (e == cudaSuccess) e = cudaMalloc(&x.hmid, nf);
+  if (e == cudaSuccess)
+    e = cudaMalloc(reinterpret_cast<void**>(&x.attn_part_o),
+                   static_cast<size_t>(hsa::kMaxAttnParts) * 256 * 128 * sizeof(float));
+  if (e == cudaSuccess)
+    e = cudaMalloc(reinterpret_cast<void**>(&x.attn_part_ml),
+                   static_cast<size_t>(hsa::kMaxAttnParts) * 256 * 2 * sizeof(float));
   if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&x.cuts), 2 * hsa::kMaxGroups * sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&x.flag), sizeof(int));
   if (e == cudaSuccess) e = cudaMemset(x.flag, 0, sizeof(int));
@@ -183,6 +189,8 @@ void hsa_destroy(hsa_ctx* ctx) {
   cudaFree(x.q);
   cudaFree(x.o);
   cudaFree(x.hmid);
+  cudaFree(x.attn_part_o);
+  cudaFree(x.attn_part_ml);
   cudaFree(x.cuts);
   cudaFree(x.flag);
   delete ctx;

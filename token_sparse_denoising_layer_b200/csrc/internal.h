@@ -16,6 +16,12 @@ constexpr int kMaxGroups = 8;
 // Bits a kernel can set in the context's device flag (read by hsa_sync_check).
 enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_INDEX = 2, DEV_BAD_SCORE = 4, DEV_BAD_GROUP = 8 };
 constexpr int kRadixBins = 256;
+// Attention work split: the units of the last, partial wave are split into
+// at most kMaxSplitParts key ranges each, and into at most kMaxAttnParts
+// parts in total (their partial results live in the context's scratch:
+// kMaxAttnParts x 256 rows x 128 fp32 = 64 MiB).
+constexpr int kMaxSplitParts = 32;
+constexpr int kMaxAttnParts = 512;
 
 struct Ctx {
   hsa_model_cfg cfg{};
@@ -32,6 +38,8 @@ struct Ctx {
   void* q = nullptr;      // bf16 [N, D] compact queries
   void* o = nullptr;      // bf16 [N, D] compact attention output
   void* hmid = nullptr;   // bf16 [N, F] compact MLP hidden
+  float* attn_part_o = nullptr;   // [kMaxAttnParts][256][128] attention partial O
+  float* attn_part_ml = nullptr;  // [kMaxAttnParts][256][2] partial (max, sum)
   uint32_t* cuts = nullptr;  // selector cut keys, 2 words per cut
   int* flag = nullptr;       // device error flag
 };

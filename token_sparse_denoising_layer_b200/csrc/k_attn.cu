@@ -64,6 +64,16 @@ struct AttnParams {
   __nv_bfloat16* o;
   int ld;            // D
   int* flag;
+  // Work decomposition.  A unit is one (pair of query tiles, head), ordered
+  // head-major.  CTAs [0, n_full) each do a whole unit; the remaining
+  // units (the last, partial wave) are each split into `split` key ranges,
+  // one CTA per range, which write unnormalised partial results that
+  // k_attn_combine merges.
+  int n_qpairs;      // units per head
+  int n_full;        // units done whole
+  int split;         // key-range parts per remaining unit
+  float* part_o;     // [part][256 rows][HD] fp32, unnormalised
+  float2* part_ml;   // [part][256 rows] (running max, row sum)
 };
 
 template <int HD>
@@ -89,10 +99,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(o_done + 2);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int q0 = blockIdx.x * (2 * kQ);
-  const int h = blockIdx.y;
+  const int nkv_all = (p.N + kKV - 1) / kKV;
+  int unit, part = -1, j0 = 0, nkv = nkv_all;
+  if (static_cast<int>(blockIdx.x) < p.n_full) {
+    unit = blockIdx.x;
+  } else {
+    part = blockIdx.x - p.n_full;
+    unit = p.n_full + part / p.split;
+    const int piece = part % p.split;
+    j0 = piece * nkv_all / p.split;
+    nkv = (piece + 1) * nkv_all / p.split - j0;  // key tiles j0 .. j0+nkv-1
+  }
+  const int q0 = (unit % p.n_qpairs) * (2 * kQ);
+  const int h = unit / p.n_qpairs;
   const int col0 = h * HD;
-  const int nkv = (p.N + kKV - 1) / kKV;
   const int ntile = (q0 + kQ < p.n) ? 2 : 1;  // second query tile empty on the last CTA
 
   if (threadIdx.x == 0) {
@@ -144,7 +164,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive_expect_tx(&k_full[s], Cfg::kTileBytes);
         for (int r = 0; r < Cfg::kRegions; ++r)
           tma_load_2d_hint(sK + s * Cfg::kTileBytes + r * Cfg::kRegionBytes, &tmK, &k_full[s],
-                           col0 + 64 * r, j * kKV, keep);
+                           col0 + 64 * r, (j0 + j) * kKV, keep);
         if (!mbar_wait(&v_empty[s], ph)) {
           ok = false;
           break;
@@ -152,7 +172,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive_expect_tx(&v_full[s], Cfg::kTileBytes);
         for (int r = 0; r < Cfg::kRegions; ++r)
           tma_load_2d_hint(sV + s * Cfg::kTileBytes + r * Cfg::kRegionBytes, &tmV, &v_full[s],
-                           col0 + 64 * r, j * kKV, keep);
+                           col0 + 64 * r, (j0 + j) * kKV, keep);
       }
     }
   } else if (warp == 1) {
@@ -239,7 +259,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         break;
       }
       tc_fence_after();
-      const int valid = p.N - j * kKV;  // keys past N are zero-filled: mask them
+      const int valid = p.N - (j0 + j) * kKV;  // keys past N are zero-filled: mask them
       // the whole S row of this tile in one TMEM load
       uint32_t sr[kKV];
       tmem_ld128(tS, sr);
@@ -291,19 +311,28 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&p_full[t]);
     }
-    // epilogue: O / l -> bf16 rows of the compact output
+    // epilogue: O / l -> bf16 rows of the compact output, or, for a key-range
+    // part, the unnormalised O with its (m, l) for k_attn_combine
     if (active && ok) {
       if (__all_sync(0xffffffffu, mbar_wait(&o_done[t], 0))) {
         tc_fence_after();
         const float inv = 1.0f / l_run;
         const int qrow = q0 + t * kQ + row;
         __nv_bfloat16* orow = p.o + static_cast<size_t>(qrow) * p.ld + col0;
+        const size_t prow = static_cast<size_t>(part) * (2 * kQ) + t * kQ + row;
+        if (part >= 0) p.part_ml[prow] = make_float2(m_run, l_run);
 #pragma unroll 1
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t r[32];
           __syncwarp();
           tmem_ld32(tO + 32 * c, r);
-          if (qrow < p.n) {
+          if (part >= 0) {
+            float4* d4 = reinterpret_cast<float4*>(p.part_o + prow * HD + 32 * c);
+#pragma unroll
+            for (int v = 0; v < 8; ++v)
+              d4[v] = make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                                  __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+          } else if (qrow < p.n) {
             uint4* d4 = reinterpret_cast<uint4*>(orow + 32 * c);
 #pragma unroll
             for (int v = 0; v < 4; ++v)
@@ -326,6 +355,44 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     tc_fence_after();
     tmem_dealloc(tmem, kTmemCols);
   }
+}
+
+// Merge the key-range parts of the split units: one warp per query row,
+// O = sum_i O_i 2^(m_i - M) / sum_i l_i 2^(m_i - M) with M = max_i m_i.
+template <int HD>
+__global__ void __launch_bounds__(256) k_attn_combine(AttnParams p) {
+  const int lane = threadIdx.x & 31;
+  const int rr = blockIdx.x * 8 + (threadIdx.x >> 5);  // row over the split units
+  const int u = blockIdx.y;                             // split unit 0..r-1
+  if (rr >= 2 * kQ) return;
+  const int unit = p.n_full + u;
+  const int q0 = (unit % p.n_qpairs) * (2 * kQ);
+  const int h = unit / p.n_qpairs;
+  const int qrow = q0 + rr;
+  if (qrow >= p.n) return;
+  float M = -INFINITY;
+  for (int i = 0; i < p.split; ++i) {
+    const size_t prow = static_cast<size_t>(u * p.split + i) * (2 * kQ) + rr;
+    M = fmaxf(M, p.part_ml[prow].x);
+  }
+  constexpr int kPer = HD / 32;  // columns per lane
+  float acc[kPer];
+#pragma unroll
+  for (int c = 0; c < kPer; ++c) acc[c] = 0.f;
+  float L = 0.f;
+  for (int i = 0; i < p.split; ++i) {
+    const size_t prow = static_cast<size_t>(u * p.split + i) * (2 * kQ) + rr;
+    const float2 ml = p.part_ml[prow];
+    const float wgt = ex2_approx(ml.x - M);
+    L += ml.y * wgt;
+    const float* po = p.part_o + prow * HD;
+#pragma unroll
+    for (int c = 0; c < kPer; ++c) acc[c] += po[lane + 32 * c] * wgt;
+  }
+  const float inv = 1.0f / L;
+  __nv_bfloat16* orow = p.o + static_cast<size_t>(qrow) * p.ld + h * HD;
+#pragma unroll
+  for (int c = 0; c < kPer; ++c) orow[lane + 32 * c] = __float2bfloat16_rn(acc[c] * inv);
 }
 
 template <int HD>
@@ -351,8 +418,33 @@ cudaError_t launch_hd(const Ctx& c, const void* q, int n, const void* kc, const 
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  const dim3 grid((n + 2 * kQ - 1) / (2 * kQ), c.cfg.H);
-  k_attn<HD><<<grid, kAttnThreads, smem, c.stream>>>(tq, tk, tv, p);
+  // Work plan: whole units fill complete waves of the SMs; the units of the
+  // last, partial wave are split along the keys so that wave is short too.
+  p.n_qpairs = (n + 2 * kQ - 1) / (2 * kQ);
+  const int units = p.n_qpairs * c.cfg.H;
+  const int nkv_all = (N + kKV - 1) / kKV;
+  const int rem = units % c.num_sms;
+  // Split each remaining unit into s key ranges, choosing s to minimise the
+  // tail's length in units of a whole wave, ceil(rem*s / SMs) / s, with a
+  // 1% charge per extra part for its prologue, partial store and combine.
+  int split = 1;
+  if (rem > 0) {
+    double best = 1.0;
+    for (int sp = 2; sp <= nkv_all && sp <= kMaxSplitParts && rem * sp <= kMaxAttnParts; ++sp) {
+      const double rounds = static_cast<double>((rem * sp + c.num_sms - 1) / c.num_sms) / sp;
+      const double cost = rounds * (1.0 + 0.01 * sp);
+      if (cost < best) best = cost, split = sp;
+    }
+  }
+  p.n_full = split > 1 ? units - rem : units;
+  p.split = split;
+  p.part_o = c.attn_part_o;
+  p.part_ml = reinterpret_cast<float2*>(c.attn_part_ml);
+  const int n_parts = (units - p.n_full) * split;
+  k_attn<HD><<<p.n_full + n_parts, kAttnThreads, smem, c.stream>>>(tq, tk, tv, p);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess || n_parts == 0) return e;
+  k_attn_combine<HD><<<dim3(2 * kQ / 8, units - p.n_full), 256, 0, c.stream>>>(p);
   return cudaGetLastError();
 }
 
