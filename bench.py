@@ -268,6 +268,80 @@ def attention_traffic():
         return None
 
 
+def _time(fn, torch, reps=10, flush=None):
+    """Median CUDA-event time (ms) of fn() on the current stream, after warm-up;
+    with `flush`, a 256 MB buffer is written between samples (cold L2)."""
+    stream = torch.cuda.current_stream()
+    for _ in range(3):
+        fn()
+    times = []
+    for r in range(reps):
+        if flush is not None:
+            flush.fill_(float(r))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    return float(np.median(times))
+
+
+def gemm_sweep(torch, abi):
+    """The four active-row GEMMs of a 1536-wide DiT layer at |A| = 32760 (plain
+    bf16 epilogue), TFLOP/s."""
+    M, D, F = 32760, 1536, 8960
+    ctx = abi.hsa_create(N=M, D=D, H=12, F=F, L=1, T=1, budgets=[1], counts=[M])
+    g = torch.Generator(device="cuda")
+    g.manual_seed(7)
+    rnd = lambda *sh: torch.randn(sh, generator=g, device="cuda").to(torch.bfloat16)
+    out = {}
+    for name, (Nc, K) in {"qkv": (3 * D, D), "out_proj": (D, D), "mlp_up": (F, D),
+                          "mlp_down": (D, F)}.items():
+        a, w = rnd(M, K), rnd(Nc, K)
+        o = torch.empty((M, Nc), dtype=torch.bfloat16, device="cuda")
+        ms = _time(lambda: abi.hsa_linear(ctx, a, M, K, w, Nc, o), torch)
+        out[name] = {"M": M, "N": Nc, "K": K, "ms": round(ms, 4),
+                     "tflops": round(2.0 * M * Nc * K / ms / 1e9, 1)}
+        del a, w, o
+    abi.hsa_sync_check(ctx)
+    ctx.close()
+    return out
+
+
+def bandwidth_sweep(torch, abi):
+    """HBM-bound row kernels at the workloads' sizes, L2 flushed between samples:
+    the standalone KV-cache scatter (dit30 and dit40 shapes) and the LN gather."""
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    res = {}
+    for name, N, D, a in (("kv_scatter_dit30_f1", 32760, 1536, 32760),
+                          ("kv_scatter_dit40_f0.25", 75600, 5120, 18900)):
+        ctx = abi.hsa_create(N=N, D=D, H=D // 128, F=64, L=1, T=1, budgets=[1], counts=[N])
+        kr = torch.randn((a, D), device="cuda").to(torch.bfloat16)
+        vr = torch.randn((a, D), device="cuda").to(torch.bfloat16)
+        kc = torch.zeros((N, D), dtype=torch.bfloat16, device="cuda")
+        vc = torch.zeros((N, D), dtype=torch.bfloat16, device="cuda")
+        idx = torch.sort(torch.randperm(N, device="cuda")[:a]).values.to(torch.int32)
+        ms = _time(lambda: abi.hsa_kv_scatter(ctx, kr, vr, idx, a, kc, vc), torch, flush=flush)
+        nbytes = 4 * a * D * 2 + 4 * a
+        res[name] = {"rows": a, "D": D, "ms": round(ms, 4), "GBps": round(nbytes / ms / 1e6, 1)}
+        abi.hsa_sync_check(ctx)
+        ctx.close()
+        del kr, vr, kc, vc
+    N, D = 32760, 1536
+    ctx = abi.hsa_create(N=N, D=D, H=12, F=64, L=1, T=1, budgets=[1], counts=[N])
+    x = torch.randn((N, D), device="cuda")
+    u = torch.empty((N, D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.arange(N, dtype=torch.int32, device="cuda")
+    ms = _time(lambda: abi.hsa_ln_gather(ctx, x, idx, N, u), torch, flush=flush)
+    nbytes = N * D * (4 + 2) + N * 4
+    res["ln_gather_dit30_f1"] = {"rows": N, "D": D, "ms": round(ms, 4),
+                                 "GBps": round(nbytes / ms / 1e6, 1)}
+    ctx.close()
+    del flush
+    return res
+
+
 def cpu_baseline(spec, n_rows=64, target_s=12.0):
     """The oracle on the host cores, on a bounded sample: one layer of the
     30-layer DiT for `n_rows` active rows against the full N = 32760 cache,
@@ -367,7 +441,9 @@ def run_ours(args, rank, world, local, pg):
     sub = {}
     if not args.quick and rank == 0:
         sub["attention"] = attention_sweep(torch, abi, synth)
+        sub["gemm"] = gemm_sweep(torch, abi)
         sub["euler"] = euler_bandwidth(torch, abi)
+        sub["bandwidth"] = bandwidth_sweep(torch, abi)
 
     result = None
     if rank == 0:
@@ -376,6 +452,10 @@ def run_ours(args, rank, world, local, pg):
         if os.path.exists(pp):
             with open(pp) as f:
                 peaks = json.load(f)
+        hbm = peaks.get("hbm_gbs", 6650.0)
+        for grp in ("euler", "bandwidth"):
+            for v in sub.get(grp, {}).values():
+                v["frac_of_hbm"] = round(v["GBps"] / hbm, 3)
         # the attention sweep times the kernel alone (10 launches back to back): burst peak
         peak_tf = peaks.get("bf16_tflops", 1590.0)
         roof = None
