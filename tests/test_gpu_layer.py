@@ -22,7 +22,8 @@ def _ctx(N, D, H, F):
 
 @pytest.mark.parametrize("M,K,Ncols", [(1, 64, 32), (128, 128, 256), (333, 256, 384),
                                        (700, 1536, 4608), (129, 512, 1536), (5, 6144, 128),
-                                       (2000, 256, 2048), (20000, 1536, 1536)])
+                                       (2000, 256, 2048), (20000, 1536, 1536),
+                                       (2300, 256, 2048), (32760, 1536, 4608)])
 def test_linear(M, K, Ncols):
     need_gpu()
     ctx = _ctx(max(M, 1), 128, 1, 64)

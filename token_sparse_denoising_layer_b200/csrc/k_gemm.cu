@@ -32,6 +32,8 @@ namespace {
 constexpr int kBM = 128;
 constexpr int kBK = 64;
 constexpr int kGemmThreads = 192;
+// relative cost per output element of a CTA-pair tile vs a 1-CTA 256-wide tile
+constexpr double kPairCost = 0.8;
 
 template <int BN>
 struct GemmCfg {
@@ -264,6 +266,212 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// ------------------------------------------------------------ CTA-pair GEMM
+// 256 x 256 output tiles computed by a cluster of two CTAs with one
+// tcgen05.mma.cta_group::2 per K-step: each CTA stages its own 128 rows of A
+// and one 128-row half of B, so a CTA moves half the B bytes of a 1-CTA
+// 128 x 256 tile through shared memory for the same MMA work.  Rank 0 issues
+// the MMAs; both CTAs load, and both run the epilogue on the 128 rows of the
+// accumulator held in their own TMEM.
+
+constexpr int kPairStages = 6;
+constexpr int kPairABytes = 128 * kBK * 2;
+constexpr int kPairBBytes = 128 * kBK * 2;
+constexpr int kPairStageBytes = kPairABytes + kPairBBytes;
+constexpr int kPairSmem = kPairStages * kPairStageBytes + 256 + 1024;
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
+    k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                EpiParams p, int n_tiles, int total_tiles) {
+  constexpr int S = kPairStages;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~static_cast<uintptr_t>(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + S * kPairABytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + S * kPairBBytes);  // used in rank 0
+  uint64_t* empty = full + S;
+  uint64_t* acc_full = empty + S;      // [2]
+  uint64_t* acc_empty = acc_full + 2;  // [2], used in rank 0
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int nk = p.Kd / kBK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 8);  // 4 epilogue warps in each CTA
+    }
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  cluster_sync();  // both CTAs' barriers initialised and TMEM allocated
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  bool ok = true;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      int it = 0;
+      for (int t = pair; t < total_tiles && ok; t += npairs) {
+        const int m0 = (t / n_tiles) * 256 + rank * 128, n0 = (t % n_tiles) * 256 + rank * 128;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(&empty[s], ((it / S) & 1) ^ 1)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_arrive_expect_tx(&full[s], 2 * kPairStageBytes);
+          const uint32_t lead = to_leader(smem_u32(&full[s]));
+          tma_load_2d_pair(sA + s * kPairABytes, &tmA, lead, kb * kBK, m0);
+          tma_load_2d_pair(sB + s * kPairBBytes, &tmB, lead, kb * kBK, n0);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16(256, 256, false, false);
+      int it = 0, lt = 0;
+      for (int t = pair; t < total_tiles && ok; t += npairs, ++lt) {
+        const int b = lt & 1;
+        if (!mbar_wait(&acc_empty[b], ((lt >> 1) & 1) ^ 1)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t acc = tmem + b * 256;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % S;
+          if (!mbar_wait(&full[s], (it / S) & 1)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = smem_u32(sA + s * kPairABytes);
+          const uint32_t b0 = smem_u32(sB + s * kPairBBytes);
+#pragma unroll
+          for (int kk = 0; kk < kBK / 16; ++kk)
+            umma_bf16_pair(acc, sdesc_sw128(a0 + kk * 32, 16, 1024),
+                           sdesc_sw128(b0 + kk * 32, 16, 1024), idesc, (kb > 0 || kk > 0) ? 1u : 0u);
+          umma_commit_pair(&empty[s], 0x3);
+        }
+        umma_commit_pair(&acc_full[b], 0x3);
+      }
+    }
+  } else {
+    const int q = warp & 3;
+    const int row = 32 * q + lane;
+    const uint32_t lead_empty0 = to_leader(smem_u32(&acc_empty[0]));
+    const uint32_t lead_empty1 = to_leader(smem_u32(&acc_empty[1]));
+    int lt = 0;
+    for (int t = pair; t < total_tiles; t += npairs, ++lt) {
+      const int b = lt & 1;
+      if (!__all_sync(0xffffffffu, mbar_wait(&acc_full[b], (lt >> 1) & 1))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int m = (t / n_tiles) * 256 + rank * 128 + row, n0 = (t % n_tiles) * 256;
+      const bool mrow = m < p.M;
+      int32_t dst_row = 0;
+      if (mrow && (p.epi == EPI_QKV || p.epi == EPI_RESID)) {
+        dst_row = __ldg(p.idx + m);
+        if (!row_ok(dst_row, p.N, p.flag)) dst_row = -1;
+      }
+      const uint32_t tbase = tmem + b * 256 + (static_cast<uint32_t>(32 * q) << 16);
+#pragma unroll 1
+      for (int c0 = 0; c0 < 256; c0 += 32) {
+        uint32_t r[32];
+        __syncwarp();
+        tmem_ld32(tbase + c0, r);
+        const int col = n0 + c0;
+        if (mrow && col < p.Ncols) switch (p.epi) {
+          case EPI_STORE:
+            store_bf16x32<false>(p.out + static_cast<size_t>(m) * p.ld_out + col, r);
+            break;
+          case EPI_GELU:
+            store_bf16x32<true>(p.out + static_cast<size_t>(m) * p.ld_out + col, r);
+            break;
+          case EPI_QKV: {
+            const int D = p.ld_out;
+            const int which = col / D;
+            const int cc = col - which * D;
+            if (which == 0) {
+              store_bf16x32<false>(p.out + static_cast<size_t>(m) * D + cc, r);
+            } else if (dst_row >= 0) {
+              __nv_bfloat16* cache = which == 1 ? p.kc : p.vc;
+              store_bf16x32<false>(cache + static_cast<size_t>(dst_row) * D + cc, r);
+            }
+            break;
+          }
+          case EPI_RESID:
+            if (dst_row >= 0) add_f32x32(p.x + static_cast<size_t>(dst_row) * p.ld_x + col, r);
+            break;
+          default:
+            break;
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(b == 0 ? lead_empty0 : lead_empty1);
+    }
+  }
+  if (!ok) atomicOr(p.flag, DEV_TIMEOUT);
+  tc_fence_before();
+  cluster_sync();  // no CTA leaves while its peer may still signal its barriers
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+cudaError_t launch_pair(const Ctx& c, const GemmArgs& a, std::string* why) {
+  CUtensorMap ta, tb;
+  if (!make_tmap_bf16(&ta, a.A, a.M, a.Kd, a.Kd, 128, why)) return cudaErrorInvalidValue;
+  if (!make_tmap_bf16(&tb, a.B, a.Ncols, a.Kd, a.Kd, 128, why)) return cudaErrorInvalidValue;
+  EpiParams p{};
+  p.M = a.M;
+  p.Ncols = a.Ncols;
+  p.Kd = a.Kd;
+  p.epi = a.epi;
+  p.out = static_cast<__nv_bfloat16*>(a.out);
+  p.ld_out = a.ld_out;
+  p.kc = static_cast<__nv_bfloat16*>(a.k_cache);
+  p.vc = static_cast<__nv_bfloat16*>(a.v_cache);
+  p.x = a.x;
+  p.ld_x = a.ld_x;
+  p.idx = a.idx;
+  p.N = a.N;
+  p.flag = c.flag;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(k_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         kPairSmem);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int n_tiles = (a.Ncols + 255) / 256;
+  const int total = n_tiles * ((a.M + 255) / 256);
+  const int pairs = total < c.num_sms / 2 ? total : c.num_sms / 2;
+  k_gemm_pair<<<2 * pairs, kGemmThreads, kPairSmem, c.stream>>>(ta, tb, p, n_tiles, total);
+  return cudaGetLastError();
+}
+
 template <int BN>
 cudaError_t launch_bn(const Ctx& c, const GemmArgs& a, std::string* why) {
   CUtensorMap ta, tb;
@@ -315,9 +523,20 @@ cudaError_t launch_gemm(const Ctx& c, const GemmArgs& a, std::string* why) {
   };
   double best = 1e300;
   int bn = 128;
+  // CTA pairs: 256 x 256 tiles over SMs/2 pairs, about 0.8x the cost per output
+  // element of a 1-CTA 256-wide tile (half the B traffic through shared memory)
+  if (a.Ncols % 256 == 0 && a.M >= 256) {
+    const int mt2 = (a.M + 255) / 256;
+    const long tiles2 = static_cast<long>(mt2) * (a.Ncols / 256);
+    const int pairs = c.num_sms / 2;
+    // a pair tile is the same work per SM as a 1-CTA 128 x 256 tile
+    const double pc = static_cast<double>((tiles2 + pairs - 1) / pairs) * 256 * kPairCost;
+    if (pc < best) best = pc, bn = -1;
+  }
   if (a.Ncols % 256 == 0 && cost(256, 1.0) < best) best = cost(256, 1.0), bn = 256;
   if (a.Ncols % 192 == 0 && cost(192, 1.03) < best) best = cost(192, 1.03), bn = 192;
   if (cost(128, 1.12) < best) best = cost(128, 1.12), bn = 128;
+  if (bn == -1) return launch_pair(c, a, why);
   if (bn == 256) return launch_bn<256>(c, a, why);
   if (bn == 192) return launch_bn<192>(c, a, why);
   return launch_bn<128>(c, a, why);
