@@ -216,6 +216,21 @@ def attention_sweep(torch, abi, synth):
                                    "tflops": round(flop / ms / 1e9, 1)}
     abi.hsa_sync_check(ctx)
     ctx.close()
+    del kc, vc, q, o
+    # the 40-layer DiT's attention shape: N = 75600 (21x45x80), 40 heads x 128
+    N, D, H = 75600, 5120, 40
+    ctx = abi.hsa_create(N=N, D=D, H=H, F=64, L=1, T=1, budgets=[1], counts=[N])
+    kc = torch.randn((N, D), generator=g, device="cuda").to(torch.bfloat16)
+    vc = torch.randn((N, D), generator=g, device="cuda").to(torch.bfloat16)
+    q = torch.randn((N, D), generator=g, device="cuda").to(torch.bfloat16)
+    o = torch.empty((N, D), dtype=torch.bfloat16, device="cuda")
+    for f in (1.0, 0.25):
+        a = int(round(f * N))
+        ms = _time(lambda: abi.hsa_attention(ctx, q, a, kc, vc, o), torch, reps=3)
+        out[f"dit40_{int(f * 100)}%"] = {"active": a, "N": N, "D": D, "ms": round(ms, 3),
+                                         "tflops": round(4.0 * a * N * D / ms / 1e9, 1)}
+    abi.hsa_sync_check(ctx)
+    ctx.close()
     return out
 
 

@@ -100,3 +100,29 @@ def test_dit30_shapes_loop_drift():
     print(f"dit30-shape loop (L=1, N=840, T=40) x_T drift vs float64 oracle: {drift:.3e}")
     assert drift <= 2e-2
     loop.close()
+
+
+def test_dit40_shapes_loop_drift():
+    """The whole loop at the 40-layer DiT's D, H, F, T, shift and budgets ({40, 10}
+    at 25/75%), with one layer and N = 210 tokens, against the float64 oracle."""
+    need_gpu()
+    spec = synth.WORKLOADS["dit40_5120"]
+    sh = synth.ModelShape(N=210, C=16, D=5120, H=40, F=13824, L=1)
+    T, budgets = spec["T"], list(spec["budgets"])
+    counts = synth.group_counts(sh.N, spec["fractions"])
+    w = synth.model_weights(sh, 4)
+    layers = [tuple(bf(lw[k]) for k in ("w_qkv", "w_o", "w_1", "w_2")) for lw in w["layers"]]
+    from token_sparse_denoising_layer_b200.loop import HsaLoop
+    loop = HsaLoop(sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]), T, budgets,
+                   counts, shift=spec["shift"])
+    x0 = synth.latent(sh.N, 16, 4)
+    g0 = synth.random_split(sh.N, counts, 4)
+    loop.reset(x0, g0)
+    loop.run(regroup=False)
+    abi.hsa_sync_check(loop.ctx)
+    xr = O.run_loop(w, x0, g0, T, budgets, counts, O.sigma_schedule(T, spec["shift"]), sh.H,
+                    regroup=False)
+    drift = float(np.linalg.norm(host(loop.x) - xr) / np.linalg.norm(xr))
+    print(f"dit40-shape loop (L=1, N=210, T=40) x_T drift vs float64 oracle: {drift:.3e}")
+    assert drift <= 2e-2
+    loop.close()
