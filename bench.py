@@ -175,16 +175,6 @@ def time_steps(loop, steps, torch, regroup=True, per_step_hook=None):
     return [a.elapsed_time(b) for a, b in ev]
 
 
-def kernels_per_step(loop, i, regroup=True):
-    """Kernel launches of one hsa_step: schedule, embed, 7 per layer, head, Euler,
-    and 3 for re-grouping when it runs."""
-    n = 4 + 7 * loop.L
-    smin = min(loop.budgets)
-    if regroup and loop.T // smin <= i < loop.T - 1:
-        n += 3 if len(loop.budgets) > 1 else 1
-    return n
-
-
 def attention_sweep(torch, abi, synth):
     """Single DiT layer, N = 32760, hidden 1536, 12 x 128 heads: attention of
     |A| = f*N queries against the full cache, f in {1, .5, .25, .1}."""
@@ -415,9 +405,10 @@ def run_ours(args, rank, world, local, pg):
     abi.hsa_sync_check(loop.ctx)
     loop.reset(x0, g0)
     barrier(pg)
-    launches = sum(kernels_per_step(loop, k % loop.T) for k in range(args.steps))
+    launches0 = abi.hsa_kernel_launches(loop.ctx)
     with ClockSampler(local) as clk:
         times = time_steps(loop, args.steps, torch)
+    launches = abi.hsa_kernel_launches(loop.ctx) - launches0
     abi.hsa_sync_check(loop.ctx)
     ms_total = max_over_ranks(float(np.sum(times)), pg, torch.device("cuda", local))
     ms_step = ms_total / args.steps

@@ -126,6 +126,9 @@ hsa_status hsa_sync_check(hsa_ctx* ctx);
  */
 hsa_status hsa_selftest_timeout(hsa_ctx* ctx, int timeout_us);
 
+/* Number of kernels this context has launched so far (host counter, no sync). */
+uint64_t hsa_kernel_launches(const hsa_ctx* ctx);
+
 /*
  * |A_i| computed on the host from the group counts ([TS] 2.1): the sum of n_k
  * over the groups active at iteration i.  Valid when g holds exactly counts[k]

@@ -98,3 +98,22 @@ def test_phase_window_loop_drift():
     d = _drift(host(loop.x), xr)
     print(f"tiny DiT with phase window m=2: x_T drift {d:.3e}")
     assert d <= 2e-2
+
+
+def test_kernel_launch_counter():
+    """The context counts the kernels it launches: per iteration schedule,
+    embed, head and Euler, and per layer LN x2, QKV, attention + part-combine,
+    out-proj, MLP up and down; re-grouping adds score, cut search and assign."""
+    need_gpu()
+    sh, T, counts, w, loop, x0, g0 = _setup()
+    loop.reset(x0, g0)
+    c0 = abi.hsa_kernel_launches(loop.ctx)
+    loop.step(0)                               # no re-grouping before i = T / s_K = 2
+    c1 = abi.hsa_kernel_launches(loop.ctx)
+    loop.step(1)
+    loop.step(2)                               # re-groups
+    c3 = abi.hsa_kernel_launches(loop.ctx)
+    abi.hsa_sync_check(loop.ctx)
+    per_step = 4 + 8 * sh.L
+    assert c1 - c0 == per_step
+    assert c3 - c1 == 2 * per_step + 3

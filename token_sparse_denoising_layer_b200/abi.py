@@ -18,7 +18,7 @@ LIB_PATH = os.path.join(PKG, "libhsa.so")
 # Every symbol the header declares, in header order.
 SYMBOLS = [
     "hsa_create", "hsa_destroy", "hsa_last_error", "hsa_set_stream", "hsa_sync_check",
-    "hsa_selftest_timeout", "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
+    "hsa_selftest_timeout", "hsa_kernel_launches", "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
     "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_linear", "hsa_kv_scatter",
     "hsa_attention", "hsa_out_proj_residual", "hsa_mlp_residual", "hsa_layer_forward",
     "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_step", "hsa_select_groups_static",
@@ -82,6 +82,7 @@ def load() -> ctypes.CDLL:
         "hsa_set_stream": (I, [P, P]),
         "hsa_sync_check": (I, [P]),
         "hsa_selftest_timeout": (I, [P, I]),
+        "hsa_kernel_launches": (ctypes.c_uint64, [P]),
         "hsa_n_active": (I, [P, I]),
         "hsa_schedule": (I, [P, I, P, P, P, P, ctypes.POINTER(I)]),
         "hsa_score": (I, [P, P, P, P]),
@@ -179,6 +180,10 @@ def hsa_sync_check(ctx: Context) -> None:
 
 def hsa_selftest_timeout(ctx: Context, timeout_us: int) -> None:
     _check(ctx.ptr, load().hsa_selftest_timeout(ctx.ptr, timeout_us))
+
+
+def hsa_kernel_launches(ctx: Context) -> int:
+    return int(load().hsa_kernel_launches(ctx.ptr))
 
 
 def hsa_n_active(ctx: Context, i: int) -> int:

@@ -227,6 +227,8 @@ hsa_status hsa_selftest_timeout(hsa_ctx* ctx, int timeout_us) {
                   "selftest_timeout");
 }
 
+uint64_t hsa_kernel_launches(const hsa_ctx* ctx) { return ctx ? ctx->c.launches : 0; }
+
 int hsa_n_active(const hsa_ctx* ctx, int i) {
   if (ctx == nullptr || i < 0 || i >= ctx->c.T) return -1;
   const Ctx& x = ctx->c;

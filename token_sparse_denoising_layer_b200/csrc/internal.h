@@ -33,6 +33,7 @@ struct Ctx {
   int device = 0;
   int num_sms = 148;
   std::string err;
+  mutable uint64_t launches = 0;  // kernels launched through this context
   // scratch (device)
   void* u = nullptr;      // bf16 [N, D] LN output of the active rows
   void* q = nullptr;      // bf16 [N, D] compact queries

@@ -442,9 +442,11 @@ cudaError_t launch_hd(const Ctx& c, const void* q, int n, const void* kc, const 
   p.part_ml = reinterpret_cast<float2*>(c.attn_part_ml);
   const int n_parts = (units - p.n_full) * split;
   k_attn<HD><<<p.n_full + n_parts, kAttnThreads, smem, c.stream>>>(tq, tk, tv, p);
+  c.launches += 1;
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess || n_parts == 0) return e;
   k_attn_combine<HD><<<dim3(2 * kQ / 8, units - p.n_full), 256, 0, c.stream>>>(p);
+  c.launches += 1;
   return cudaGetLastError();
 }
 

@@ -469,6 +469,7 @@ cudaError_t launch_pair(const Ctx& c, const GemmArgs& a, std::string* why) {
   const int total = n_tiles * ((a.M + 255) / 256);
   const int pairs = total < c.num_sms / 2 ? total : c.num_sms / 2;
   k_gemm_pair<<<2 * pairs, kGemmThreads, kPairSmem, c.stream>>>(ta, tb, p, n_tiles, total);
+  c.launches += 1;
   return cudaGetLastError();
 }
 
@@ -502,6 +503,7 @@ cudaError_t launch_bn(const Ctx& c, const GemmArgs& a, std::string* why) {
   const int total = n_tiles * ((a.M + kBM - 1) / kBM);
   const int grid = total < c.num_sms ? total : c.num_sms;
   k_gemm<BN><<<grid, kGemmThreads, smem, c.stream>>>(ta, tb, p, n_tiles, total);
+  c.launches += 1;
   return cudaGetLastError();
 }
 

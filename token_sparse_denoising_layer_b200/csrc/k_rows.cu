@@ -123,6 +123,7 @@ cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, i
     case 16: k_ln_gather<16><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
     default: k_ln_gather_any<<<grid, block, 0, c.stream>>>(x, idx, n, N, D, uo, c.flag); break;
   }
+  c.launches += 1;
   return cudaGetLastError();
 }
 
@@ -157,6 +158,7 @@ cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_ro
   k_kv_scatter<<<static_cast<unsigned>(blocks), 256, 0, c.stream>>>(
       static_cast<const uint4*>(k_rows), static_cast<const uint4*>(v_rows), idx, n, c.cfg.N, vpr,
       static_cast<uint4*>(kc), static_cast<uint4*>(vc), c.flag);
+  c.launches += 1;
   return cudaGetLastError();
 }
 
@@ -208,6 +210,7 @@ cudaError_t launch_embed(const Ctx& c, const float* w_in, const float* x_lat, co
   const size_t total = static_cast<size_t>(n) * (c.cfg.D / 4);
   k_embed<<<static_cast<unsigned>((total + 255) / 256), 256, 0, c.stream>>>(
       w_in, x_lat, idx, n, c.cfg.N, c.cfg.D, h, c.flag);
+  c.launches += 1;
   return cudaGetLastError();
 }
 
@@ -269,6 +272,7 @@ cudaError_t launch_head(const Ctx& c, const float* w_head, const float* h, const
                         int n, float* v_fresh) {
   if (n <= 0) return cudaSuccess;
   k_head<<<(n + 7) / 8, 256, 0, c.stream>>>(w_head, h, idx, n, c.cfg.N, c.cfg.D, v_fresh, c.flag);
+  c.launches += 1;
   return cudaGetLastError();
 }
 

@@ -140,6 +140,7 @@ cudaError_t launch_schedule(const Ctx& c, int i, const uint8_t* g, uint8_t* mask
   p.N = c.cfg.N;
   const int blocks = (c.cfg.N + kSchedChunk - 1) / kSchedChunk;
   k_schedule<<<blocks, kSchedThreads, 0, c.stream>>>(g, mask, idx, n_dev, p, c.flag);
+  c.launches += 1;
   return cudaGetLastError();
 }
 
@@ -181,6 +182,7 @@ cudaError_t launch_score(const Ctx& c, const float* v_prev, const float* v_cur, 
   k_score<<<(N + 255) / 256, 256, 0, c.stream>>>(reinterpret_cast<const float4*>(v_prev),
                                                  reinterpret_cast<const float4*>(v_cur), score, N,
                                                  c.flag);
+  c.launches += 1;
   return cudaGetLastError();
 }
 
@@ -308,6 +310,7 @@ cudaError_t launch_select(const Ctx& c, const float* score, uint8_t* g) {
     cp.rank[j] = acc;
   }
   k_radix_cut<<<ncut, kSelThreads, 0, c.stream>>>(score, N, cp, c.cuts, c.flag);
+  c.launches += 2;  // with k_assign below
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   k_assign<<<(N + 255) / 256, 256, 0, c.stream>>>(score, c.cuts, ncut, g, N);
@@ -355,6 +358,7 @@ __global__ void k_selftest_timeout(uint64_t limit_ns, int* flag) {
 
 cudaError_t launch_selftest_timeout(const Ctx& c, uint64_t limit_ns) {
   k_selftest_timeout<<<1, 1, 0, c.stream>>>(limit_ns, c.flag);
+  c.launches += 1;
   return cudaGetLastError();
 }
 
@@ -397,6 +401,7 @@ cudaError_t launch_euler(const Ctx& c, float* x, float* v_hat, float* v_hat_prev
       reinterpret_cast<float4*>(x), reinterpret_cast<float4*>(v_hat),
       reinterpret_cast<float4*>(v_hat_prev), reinterpret_cast<const float4*>(v_fresh), mask, s0,
       s1, n4);
+  c.launches += 1;
   return cudaGetLastError();
 }
 
