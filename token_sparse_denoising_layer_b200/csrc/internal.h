@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
 #include <string>
 
 #include "../../include/hsa.h"
@@ -51,6 +52,17 @@ __device__ __forceinline__ bool row_ok(int32_t r, int N, int* flag) {
   if (static_cast<uint32_t>(r) < static_cast<uint32_t>(N)) return true;
   atomicOr(flag, DEV_BAD_INDEX);
   return false;
+}
+
+// Raise a kernel's dynamic shared-memory limit, once per device (bit d of `done`).
+template <typename Kernel>
+cudaError_t ensure_smem_limit(Kernel* kernel, int bytes, int device, std::atomic<uint64_t>& done) {
+  const uint64_t bit = 1ull << (device & 63);
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  const cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
 }
 
 // ---- launchers (return cudaGetLastError() of the launch)

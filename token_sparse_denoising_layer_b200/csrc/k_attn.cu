@@ -411,12 +411,10 @@ cudaError_t launch_hd(const Ctx& c, const void* q, int n, const void* kc, const 
   p.ld = D;
   p.flag = c.flag;
   constexpr int smem = AttnCfg<HD>::kSmem;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e =
-        cudaFuncSetAttribute(k_attn<HD>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static std::atomic<uint64_t> smem_set{0};  // per device
+  {
+    const cudaError_t e = ensure_smem_limit(k_attn<HD>, smem, c.device, smem_set);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   // Work plan: whole units fill complete waves of the SMs; the units of the
   // last, partial wave are split along the keys so that wave is short too.

@@ -458,12 +458,10 @@ cudaError_t launch_pair(const Ctx& c, const GemmArgs& a, std::string* why) {
   p.idx = a.idx;
   p.N = a.N;
   p.flag = c.flag;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm_pair, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         kPairSmem);
+  static std::atomic<uint64_t> smem_set{0};  // per device
+  {
+    const cudaError_t e = ensure_smem_limit(k_gemm_pair, kPairSmem, c.device, smem_set);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   const int n_tiles = (a.Ncols + 255) / 256;
   const int total = n_tiles * ((a.M + 255) / 256);
@@ -493,11 +491,10 @@ cudaError_t launch_bn(const Ctx& c, const GemmArgs& a, std::string* why) {
   p.N = a.N;
   p.flag = c.flag;
   constexpr int smem = GemmCfg<BN>::kSmem;
-  static bool attr_set = false;  // one device per process is the supported use
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(k_gemm<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static std::atomic<uint64_t> smem_set{0};  // per device
+  {
+    const cudaError_t e = ensure_smem_limit(k_gemm<BN>, smem, c.device, smem_set);
     if (e != cudaSuccess) return e;
-    attr_set = true;
   }
   const int n_tiles = (a.Ncols + BN - 1) / BN;
   const int total = n_tiles * ((a.M + kBM - 1) / kBM);

@@ -18,7 +18,6 @@
 #include <stdint.h>
 
 #include <mutex>
-#include <string>
 
 #include "../../include/hsa.h"
 #include "internal.h"
@@ -37,23 +36,19 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
 
-// Errors are reported by status code only: this entry point has no context
-// to hold a message.
-hsa_status static_fail(hsa_status st, const std::string&) { return st; }
-
 // Device address of the scratch array on the current device, looked up once
 // per device.  In host code the array's name is only a host-side stand-in.
+// Errors are reported by status code only: this entry point has no context to
+// hold a message.
 hsa_status scratch_address(void** out) {
   int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return static_fail(HSA_ERR_CUDA, std::string("cudaGetDevice: ") + cudaGetErrorString(e));
-  if (dev < 0 || dev >= kMaxDevices) return static_fail(HSA_ERR_INVALID_ARG, "device ordinal out of range");
+  if (cudaGetDevice(&dev) != cudaSuccess) return HSA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return HSA_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
   if (g_scratch_addr[dev] == nullptr) {
     void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_select_scratch);
-    if (e != cudaSuccess || p == nullptr)
-      return static_fail(HSA_ERR_CUDA, std::string("cudaGetSymbolAddress: ") + cudaGetErrorString(e));
+    if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || p == nullptr)
+      return HSA_ERR_CUDA;
     g_scratch_addr[dev] = p;
   }
   *out = g_scratch_addr[dev];
@@ -68,21 +63,15 @@ extern "C" {
 
 hsa_status hsa_select_groups_static(const float* v_prev, const float* v_cur, int N,
                                     const int* counts, int K, uint8_t* g, void* stream) {
-  if (N > kStaticMaxN)
-    return static_fail(HSA_ERR_SCRATCH_LIMIT,
-                       "N = " + std::to_string(N) + " is outside [1, " +
-                           std::to_string(kStaticMaxN) + "], the size of the static scratch");
-  if (N < 1) return static_fail(HSA_ERR_INVALID_ARG, "N must be >= 1");
-  if (K < 1 || K > hsa::kMaxGroups) return static_fail(HSA_ERR_INVALID_ARG, "K must be in [1, 8]");
-  if (counts == nullptr) return static_fail(HSA_ERR_INVALID_ARG, "counts is NULL");
+  if (N > kStaticMaxN) return HSA_ERR_SCRATCH_LIMIT;  // beyond the static scratch
+  if (N < 1 || K < 1 || K > hsa::kMaxGroups || counts == nullptr) return HSA_ERR_INVALID_ARG;
   long long total = 0;
   for (int k = 0; k < K; ++k) {
-    if (counts[k] < 0) return static_fail(HSA_ERR_BUDGET, "group counts must be >= 0");
+    if (counts[k] < 0) return HSA_ERR_BUDGET;
     total += counts[k];
   }
-  if (total != N) return static_fail(HSA_ERR_BUDGET, "group counts must sum to N");
-  if (!aligned16(v_prev) || !aligned16(v_cur) || !aligned16(g))
-    return static_fail(HSA_ERR_INVALID_ARG, "v_prev, v_cur and g must be non-NULL and 16-byte aligned");
+  if (total != N) return HSA_ERR_BUDGET;  // group counts must sum to N
+  if (!aligned16(v_prev) || !aligned16(v_cur) || !aligned16(g)) return HSA_ERR_INVALID_ARG;
   void* base = nullptr;
   if (hsa_status st = scratch_address(&base)) return st;
   auto* bytes = static_cast<unsigned char*>(base);
@@ -94,8 +83,7 @@ hsa_status hsa_select_groups_static(const float* v_prev, const float* v_cur, int
   cudaError_t e = cudaMemsetAsync(flag, 0, sizeof(int), s);
   if (e == cudaSuccess)
     e = hsa::launch_select_groups_raw(s, v_prev, v_cur, N, counts, K, score, cuts, g, flag);
-  if (e != cudaSuccess) return static_fail(HSA_ERR_CUDA, std::string("launch: ") + cudaGetErrorString(e));
-  return HSA_OK;
+  return e == cudaSuccess ? HSA_OK : HSA_ERR_CUDA;
 }
 
 }  // extern "C"
