@@ -237,7 +237,8 @@ def attention(q: np.ndarray, k_cache: np.ndarray, v_cache: np.ndarray, H: int,
 
 def layer_forward(w: Dict[str, np.ndarray], x: np.ndarray, idx: np.ndarray,
                   k_cache: np.ndarray, v_cache: np.ndarray, H: int,
-                  emulate_bf16: bool = False, trace: Optional[dict] = None) -> None:
+                  emulate_bf16: bool = False, trace: Optional[dict] = None,
+                  mod: Optional[np.ndarray] = None, cross: Optional[dict] = None) -> None:
     """One transformer block on the active set only ([TS] 2.2), in place.
 
     1. Only A_i goes through the QKV projection (step 1).
@@ -251,11 +252,24 @@ def layer_forward(w: Dict[str, np.ndarray], x: np.ndarray, idx: np.ndarray,
     Linear layout [out, in].  x is float [N, D]; k_cache, v_cache are float
     [N, D] (H heads of d = D/H).  ``emulate_bf16`` rounds at the points a bf16
     kernel stores: LN outputs, Q/K/V, probabilities, attention output, GELU output.
+
+    Conditioning of a real video DiT (reading; [TS] 2.2 step 4 says skipped
+    tokens incur no cross-attention, so both act on A_i only):
+    ``mod`` [6, D] = (shift_a, scale_a, gate_a, shift_m, scale_m, gate_m), the
+    timestep modulation shared by all active tokens at this iteration:
+    LN(x)*(1 + scale) + shift before the attention / MLP branch, and the branch
+    output multiplied by its gate.  ``cross`` = {w_q, w_o, k_txt, v_txt}: after
+    self-attention, x += W_oc Attn(LN(x) W_qc^T, k_txt, v_txt) against the text
+    tokens' keys and values (no cache: they are fixed for the whole run).
     """
     rb = bf16 if emulate_bf16 else (lambda t: t)
     D = x.shape[1]
     xa = np.asarray(x[idx], dtype=np.float64)
-    u = rb(layer_norm(xa))
+    m = None if mod is None else np.asarray(mod, dtype=np.float64)
+    u = layer_norm(xa)
+    if m is not None:
+        u = u * (1.0 + m[1]) + m[0]
+    u = rb(u)
     qkv = u @ np.asarray(w["w_qkv"], dtype=np.float64).T
     q = rb(qkv[:, :D])
     k = rb(qkv[:, D:2 * D])
@@ -263,13 +277,24 @@ def layer_forward(w: Dict[str, np.ndarray], x: np.ndarray, idx: np.ndarray,
     k_cache[idx] = k
     v_cache[idx] = v
     o = attention(q, k_cache, v_cache, H, emulate_bf16)
-    xa = xa + o @ np.asarray(w["w_o"], dtype=np.float64).T
-    u2 = rb(layer_norm(xa))
+    branch = o @ np.asarray(w["w_o"], dtype=np.float64).T
+    xa = xa + (branch if m is None else m[2] * branch)
+    oc = None
+    if cross is not None:
+        uc = rb(layer_norm(xa))
+        qc = rb(uc @ np.asarray(cross["w_q"], dtype=np.float64).T)
+        oc = attention(qc, cross["k_txt"], cross["v_txt"], H, emulate_bf16)
+        xa = xa + oc @ np.asarray(cross["w_o"], dtype=np.float64).T
+    u2 = layer_norm(xa)
+    if m is not None:
+        u2 = u2 * (1.0 + m[4]) + m[3]
+    u2 = rb(u2)
     hmid = rb(gelu(u2 @ np.asarray(w["w_1"], dtype=np.float64).T))
-    xa = xa + hmid @ np.asarray(w["w_2"], dtype=np.float64).T
+    branch = hmid @ np.asarray(w["w_2"], dtype=np.float64).T
+    xa = xa + (branch if m is None else m[5] * branch)
     x[idx] = xa
     if trace is not None:
-        trace.update(q=q, k=k, v=v, o=o, u=u, u2=u2, hmid=hmid)
+        trace.update(q=q, k=k, v=v, o=o, u=u, u2=u2, hmid=hmid, oc=oc)
 
 
 def embed(w_in: np.ndarray, x_lat: np.ndarray) -> np.ndarray:

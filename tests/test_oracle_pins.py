@@ -343,6 +343,72 @@ def test_refreshed_cache_gives_dense_attention():
     assert np.allclose(tr2["o"], dense[:5], atol=1e-12)
 
 
+def test_conditioning_neutral_modulation_is_the_plain_block():
+    """shift = scale = 0 and gate = 1 leave the block unchanged, bit for bit."""
+    N, D, H, F = 9, 8, 2, 16
+    w = {k: v.astype(np.float64) for k, v in synth.layer_weights(D, F, 8).items()}
+    x = synth.hidden_rows(N, D, 8).astype(np.float64)
+    idx = np.array([0, 3, 4, 8], dtype=np.int32)
+    m = np.zeros((6, D))
+    m[2] = m[5] = 1.0
+    a, b = x.copy(), x.copy()
+    O.layer_forward(w, a, idx, np.zeros((N, D)), np.zeros((N, D)), H)
+    O.layer_forward(w, b, idx, np.zeros((N, D)), np.zeros((N, D)), H, mod=m)
+    assert (a == b).all()
+
+
+def test_conditioning_zero_gates_remove_their_branch():
+    """gate_a = gate_m = 0: the block only updates the caches; x is unchanged.
+    gate_m = 0 alone: x gets exactly the (modulated) attention branch."""
+    N, D, H, F = 9, 8, 2, 16
+    w = {k: v.astype(np.float64) for k, v in synth.layer_weights(D, F, 9).items()}
+    x = synth.hidden_rows(N, D, 9).astype(np.float64)
+    idx = np.array([1, 2, 7], dtype=np.int32)
+    m = synth.modulation(D, 9).astype(np.float64)
+    m[2] = 0.0
+    m[5] = 0.0
+    xx = x.copy()
+    O.layer_forward(w, xx, idx, np.zeros((N, D)), np.zeros((N, D)), H, mod=m)
+    assert (xx == x).all()
+    m2 = synth.modulation(D, 9).astype(np.float64)
+    m2[5] = 0.0
+    xx = x.copy()
+    kc, vc = np.zeros((N, D)), np.zeros((N, D))
+    tr = {}
+    O.layer_forward(w, xx, idx, kc, vc, H, mod=m2, trace=tr)
+    want = x[idx] + m2[2] * (tr["o"] @ w["w_o"].T)
+    assert np.allclose(xx[idx], want, atol=1e-12)
+    # the modulated LN input: per-channel affine map of the normalised rows
+    assert np.allclose(tr["u"], O.layer_norm(x[idx]) * (1 + m2[1]) + m2[0], atol=1e-12)
+
+
+def test_cross_attention_textbook_and_closed_form():
+    """Cross-attention of the active queries against the text tokens: equal to a
+    textbook loop computation, and with identical text keys to the mean of the
+    text values."""
+    N, D, H, F, T = 6, 8, 2, 16, 5
+    w = {k: v.astype(np.float64) for k, v in synth.layer_weights(D, F, 10).items()}
+    c = {k: v.astype(np.float64) for k, v in synth.cross_attention_weights(D, T, 10).items()}
+    x = synth.hidden_rows(N, D, 10).astype(np.float64)
+    idx = np.array([0, 2, 5], dtype=np.int32)
+    kc, vc = np.zeros((N, D)), np.zeros((N, D))
+    tr = {}
+    xx = x.copy()
+    O.layer_forward(w, xx, idx, kc, vc, H, trace=tr, cross=c)
+    # textbook: rebuild x after self-attention, then the cross branch with loops
+    x1 = x[idx] + tr["o"] @ w["w_o"].T
+    lin = lambda W, v: [math.fsum(W[o][t] * v[t] for t in range(len(v))) for o in range(len(W))]
+    qc = [lin(c["w_q"].tolist(), _ln_loops(list(r))) for r in x1]
+    oc = _attn_loops(qc, c["k_txt"].tolist(), c["v_txt"].tolist(), H)
+    assert np.allclose(tr["oc"], np.array(oc), atol=1e-12)
+    # identical keys: every query sees the mean of the text values
+    c2 = dict(c)
+    c2["k_txt"] = np.tile(c["k_txt"][:1], (T, 1))
+    tr2 = {}
+    O.layer_forward(w, x.copy(), idx, np.zeros((N, D)), np.zeros((N, D)), H, trace=tr2, cross=c2)
+    assert np.allclose(tr2["oc"], np.tile(c["v_txt"].mean(axis=0), (len(idx), 1)), atol=1e-12)
+
+
 # ---------------------------------------------------------------- cached Euler (2.3)
 
 def test_euler_telescoping_closed_form():

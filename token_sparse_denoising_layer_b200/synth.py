@@ -36,6 +36,8 @@ __all__ = [
     "random_active_set",
     "attention_inputs",
     "score_buffer",
+    "modulation",
+    "cross_attention_weights",
 ]
 
 
@@ -246,3 +248,23 @@ def device_layer_weights(D: int, F: int, seed: int, device="cuda"):
                 * (1.0 / np.sqrt(i))).to(torch.bfloat16)
 
     return lin(3 * D, D), lin(D, D), lin(F, D), lin(D, F)
+
+
+def modulation(D: int, seed: int, spread: float = 0.5) -> np.ndarray:
+    """Timestep modulation vectors [6, D] float32: (shift, scale, gate) for the
+    attention branch, then for the MLP branch; shifts/scales ~ spread*N(0,1),
+    gates ~ 1 + spread*N(0,1)."""
+    r = rng(seed + 29)
+    m = (r.standard_normal((6, D)) * spread).astype(np.float32)
+    m[2] += 1.0
+    m[5] += 1.0
+    return m
+
+
+def cross_attention_weights(D: int, n_txt: int, seed: int) -> Dict[str, np.ndarray]:
+    """Text cross-attention: w_q, w_o [D, D] ~ N(0, 1/D) and the text tokens'
+    keys and values k_txt, v_txt [n_txt, D] ~ N(0, 1), all bf16 values as float32."""
+    r = rng(seed + 31)
+    return {"w_q": bf16_round(_linear(r, D, D)), "w_o": bf16_round(_linear(r, D, D)),
+            "k_txt": bf16_round(r.standard_normal((n_txt, D), dtype=np.float32)),
+            "v_txt": bf16_round(r.standard_normal((n_txt, D), dtype=np.float32))}
