@@ -347,6 +347,36 @@ def bandwidth_sweep(torch, abi):
     return res
 
 
+def conditioned_layer(torch, abi):
+    """One 1536-wide DiT layer (N = 32760, F = 8960) with 40% of the tokens
+    active: the plain block against the conditioned one (timestep modulation
+    plus cross-attention to 512 text tokens), ms per layer."""
+    N, D, H, F, a, n_txt = 32760, 1536, 12, 8960, 13104, 512
+    ctx = abi.hsa_create(N=N, D=D, H=H, F=F, L=1, T=1, budgets=[1], counts=[N])
+    g = torch.Generator(device="cuda")
+    g.manual_seed(11)
+    rnd = lambda *sh, s=1.0: (torch.randn(sh, generator=g, device="cuda") * s).to(torch.bfloat16)
+    lw = abi.layer_weights(rnd(3 * D, D, s=D ** -0.5), rnd(D, D, s=D ** -0.5),
+                           rnd(F, D, s=D ** -0.5), rnd(D, F, s=F ** -0.5))
+    xa = abi.cross_attn(rnd(D, D, s=D ** -0.5), rnd(D, D, s=D ** -0.5), rnd(n_txt, D),
+                        rnd(n_txt, D), n_txt)
+    mod = torch.randn((6, D), generator=g, device="cuda") * 0.5
+    mod[2] += 1.0
+    mod[5] += 1.0
+    x = torch.randn((N, D), generator=g, device="cuda")
+    kc, vc = rnd(N, D), rnd(N, D)
+    idx = torch.sort(torch.randperm(N, generator=g, device="cuda")[:a]).values.to(torch.int32)
+    plain = _time(lambda: abi.hsa_layer_forward(ctx, lw, x, idx, a, kc, vc), torch)
+    cond = _time(lambda: abi.hsa_layer_forward_cond(ctx, lw, mod, xa, x, idx, a, kc, vc), torch)
+    abi.hsa_sync_check(ctx)
+    ctx.close()
+    # cross-attention adds LN + a [a, D] x [D, D] projection twice + attention over n_txt keys
+    extra_flop = 2 * 2.0 * a * D * D + 4.0 * a * n_txt * D
+    return {"active": a, "n_txt": n_txt, "plain_ms": round(plain, 4), "cond_ms": round(cond, 4),
+            "extra_ms": round(cond - plain, 4),
+            "extra_tflops": round(extra_flop / max(cond - plain, 1e-6) / 1e9, 1)}
+
+
 def cpu_baseline(spec, n_rows=64, target_s=12.0):
     """The oracle on the host cores, on a bounded sample: one layer of the
     30-layer DiT for `n_rows` active rows against the full N = 32760 cache,
@@ -450,6 +480,7 @@ def run_ours(args, rank, world, local, pg):
         sub["gemm"] = gemm_sweep(torch, abi)
         sub["euler"] = euler_bandwidth(torch, abi)
         sub["bandwidth"] = bandwidth_sweep(torch, abi)
+        sub["conditioned_layer"] = conditioned_layer(torch, abi)
 
     result = None
     if rank == 0:

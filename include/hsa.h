@@ -215,6 +215,17 @@ hsa_status hsa_attention(hsa_ctx* ctx, const void* q, int n, const void* k_cache
                          const void* v_cache, void* o);
 
 /*
+ * The same attention against an explicit set of n_kv key/value rows, e.g. the
+ * text tokens of cross-attention ([TS] 2.2 step 4 names cross-attention as
+ * work that skipped tokens do not incur): o[m] = softmax(q[m] K^T / sqrt(d)) V
+ * per head over the n_kv rows.
+ *   q (device) bf16 [n, D];  k, v (device) bf16 [n_kv, D];  o (device) bf16 [n, D] out.
+ * HSA_ERR_SHAPE if n_kv < 1.
+ */
+hsa_status hsa_attention_kv(hsa_ctx* ctx, const void* q, int n, const void* k, const void* v,
+                            int n_kv, void* o);
+
+/*
  * Out-projection on the active rows, added into the residual rows
  * ([TS] 2.2 step 4): x[idx[m]] += o[m] W_o^T.
  *   w_o (device) bf16 [D, D];  o (device) bf16 [n, D];  x (device) fp32 [N, D] in/out.
@@ -241,6 +252,34 @@ hsa_status hsa_mlp_residual(hsa_ctx* ctx, const void* w_1, const void* w_2, floa
  */
 hsa_status hsa_layer_forward(hsa_ctx* ctx, const hsa_layer_weights* w, float* x,
                              const int32_t* idx, int n, void* k_cache, void* v_cache);
+
+/* Text cross-attention of a conditioned block: its weights and the text
+ * tokens' keys and values, fixed for the whole sampling run. */
+typedef struct {
+  const void* w_q;    /* (device) bf16 [D, D] query projection */
+  const void* w_o;    /* (device) bf16 [D, D] output projection */
+  const void* k_txt;  /* (device) bf16 [n_txt, D] */
+  const void* v_txt;  /* (device) bf16 [n_txt, D] */
+  int n_txt;          /* >= 1 */
+} hsa_cross_attn;
+
+/*
+ * A conditioned block on the active set.  The pages name timestep conditioning
+ * and text cross-attention only as work skipped tokens do not incur ([TS] 2.2
+ * step 4) and give no architecture, so this follows the usual video-DiT form:
+ *   u   = LN(x) * (1 + scale_a) + shift_a;  QKV, K/V into the caches, attention
+ *         over all N cached rows;  x += gate_a * (o W_o^T)
+ *   x  += W_oc Attn(LN(x) W_qc^T, k_txt, v_txt)            (if xa != NULL)
+ *   u2  = LN(x) * (1 + scale_m) + shift_m;  x += gate_m * (GELU(u2 W_1^T) W_2^T)
+ * with mod (device, fp32 [6, D], 16-byte aligned) holding the rows
+ * shift_a, scale_a, gate_a, shift_m, scale_m, gate_m of this iteration.
+ * mod == NULL and xa == NULL is hsa_layer_forward.  Only rows idx of x and of
+ * the caches change.  Errors as hsa_layer_forward; HSA_ERR_SHAPE if
+ * xa->n_txt < 1, HSA_ERR_INVALID_ARG for a NULL or misaligned pointer.
+ */
+hsa_status hsa_layer_forward_cond(hsa_ctx* ctx, const hsa_layer_weights* w, const float* mod,
+                                  const hsa_cross_attn* xa, float* x, const int32_t* idx, int n,
+                                  void* k_cache, void* v_cache);
 
 /*
  * Embed the active latent rows: h[idx[m]] = x_lat[idx[m]] W_in^T.

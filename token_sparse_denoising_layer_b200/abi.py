@@ -20,8 +20,8 @@ SYMBOLS = [
     "hsa_create", "hsa_destroy", "hsa_last_error", "hsa_set_stream", "hsa_sync_check",
     "hsa_selftest_timeout", "hsa_kernel_launches", "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
     "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_linear", "hsa_kv_scatter",
-    "hsa_attention", "hsa_out_proj_residual", "hsa_mlp_residual", "hsa_layer_forward",
-    "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_step", "hsa_select_groups_static",
+    "hsa_attention", "hsa_attention_kv", "hsa_out_proj_residual", "hsa_mlp_residual",
+    "hsa_layer_forward", "hsa_layer_forward_cond", "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_step", "hsa_select_groups_static",
 ]
 
 STATUS = {0: "HSA_OK", 1: "HSA_ERR_INVALID_ARG", 2: "HSA_ERR_BUDGET", 3: "HSA_ERR_SHAPE",
@@ -45,6 +45,11 @@ class hsa_model_cfg(ctypes.Structure):
 class hsa_layer_weights(ctypes.Structure):
     _fields_ = [("w_qkv", ctypes.c_void_p), ("w_o", ctypes.c_void_p),
                 ("w_1", ctypes.c_void_p), ("w_2", ctypes.c_void_p)]
+
+
+class hsa_cross_attn(ctypes.Structure):
+    _fields_ = [("w_q", ctypes.c_void_p), ("w_o", ctypes.c_void_p), ("k_txt", ctypes.c_void_p),
+                ("v_txt", ctypes.c_void_p), ("n_txt", ctypes.c_int)]
 
 
 class hsa_model_weights(ctypes.Structure):
@@ -93,9 +98,12 @@ def load() -> ctypes.CDLL:
         "hsa_linear": (I, [P, P, I, I, P, I, P]),
         "hsa_kv_scatter": (I, [P, P, P, P, I, P, P]),
         "hsa_attention": (I, [P, P, I, P, P, P]),
+        "hsa_attention_kv": (I, [P, P, I, P, P, I, P]),
         "hsa_out_proj_residual": (I, [P, P, P, P, I, P]),
         "hsa_mlp_residual": (I, [P, P, P, P, P, I]),
         "hsa_layer_forward": (I, [P, ctypes.POINTER(hsa_layer_weights), P, P, I, P, P]),
+        "hsa_layer_forward_cond": (I, [P, ctypes.POINTER(hsa_layer_weights), P,
+                                       ctypes.POINTER(hsa_cross_attn), P, P, I, P, P]),
         "hsa_embed": (I, [P, P, P, P, I, P]),
         "hsa_head": (I, [P, P, P, P, I, P]),
         "hsa_euler_step": (I, [P, P, P, P, P, P, F, F]),
@@ -231,6 +239,10 @@ def hsa_attention(ctx: Context, q, n: int, k_cache, v_cache, o) -> None:
     _check(ctx.ptr, load().hsa_attention(ctx.ptr, _p(q), n, _p(k_cache), _p(v_cache), _p(o)))
 
 
+def hsa_attention_kv(ctx: Context, q, n: int, k, v, n_kv: int, o) -> None:
+    _check(ctx.ptr, load().hsa_attention_kv(ctx.ptr, _p(q), n, _p(k), _p(v), n_kv, _p(o)))
+
+
 def hsa_out_proj_residual(ctx: Context, w_o, o, idx, n: int, x) -> None:
     _check(ctx.ptr, load().hsa_out_proj_residual(ctx.ptr, _p(w_o), _p(o), _p(idx), n, _p(x)))
 
@@ -249,6 +261,22 @@ def layer_weights(w_qkv, w_o, w_1, w_2) -> hsa_layer_weights:
 def hsa_layer_forward(ctx: Context, w: hsa_layer_weights, x, idx, n: int, k_cache, v_cache) -> None:
     _check(ctx.ptr, load().hsa_layer_forward(ctx.ptr, ctypes.byref(w), _p(x), _p(idx), n,
                                              _p(k_cache), _p(v_cache)))
+
+
+def cross_attn(w_q, w_o, k_txt, v_txt, n_txt: int) -> hsa_cross_attn:
+    """The struct holds raw device addresses, so it also keeps the tensors alive."""
+    s = hsa_cross_attn(_p(w_q), _p(w_o), _p(k_txt), _p(v_txt), n_txt)
+    s._keep = (w_q, w_o, k_txt, v_txt)
+    return s
+
+
+def hsa_layer_forward_cond(ctx: Context, w: hsa_layer_weights, mod, xa, x, idx, n: int, k_cache,
+                           v_cache) -> None:
+    """mod: device fp32 [6, D] or None;  xa: hsa_cross_attn or None."""
+    _check(ctx.ptr, load().hsa_layer_forward_cond(
+        ctx.ptr, ctypes.byref(w), _p(mod) if mod is not None else None,
+        ctypes.byref(xa) if xa is not None else None, _p(x), _p(idx), n, _p(k_cache),
+        _p(v_cache)))
 
 
 def hsa_embed(ctx: Context, w_in, x_lat, idx, n: int, h) -> None:

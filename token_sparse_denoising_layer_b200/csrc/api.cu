@@ -357,47 +357,55 @@ hsa_status hsa_attention(hsa_ctx* ctx, const void* q, int n, const void* k_cache
   HSA_CHECK_PTR(ctx, v_cache);
   HSA_CHECK_PTR(ctx, o);
   std::string why;
-  return launched(ctx, hsa::launch_attention(ctx->c, q, n, k_cache, v_cache, o, &why), "attention",
+  return launched(ctx,
+                  hsa::launch_attention(ctx->c, q, n, k_cache, v_cache, ctx->c.cfg.N, o, &why),
+                  "attention", why);
+}
+
+hsa_status hsa_attention_kv(hsa_ctx* ctx, const void* q, int n, const void* k, const void* v,
+                            int n_kv, void* o) {
+  HSA_CHECK_CTX(ctx);
+  if (hsa_status st = check_n(ctx, n)) return st;
+  if (n_kv <= 0) return fail(ctx, HSA_ERR_SHAPE, "attention_kv needs n_kv >= 1");
+  if (n == 0) return HSA_OK;
+  HSA_CHECK_PTR(ctx, q);
+  HSA_CHECK_PTR(ctx, k);
+  HSA_CHECK_PTR(ctx, v);
+  HSA_CHECK_PTR(ctx, o);
+  std::string why;
+  return launched(ctx, hsa::launch_attention(ctx->c, q, n, k, v, n_kv, o, &why), "attention_kv",
                   why);
 }
 
-hsa_status hsa_out_proj_residual(hsa_ctx* ctx, const void* w_o, const void* o,
-                                 const int32_t* idx, int n, float* x) {
-  HSA_CHECK_CTX(ctx);
-  if (hsa_status st = check_n(ctx, n)) return st;
-  if (n == 0) return HSA_OK;
-  HSA_CHECK_PTR(ctx, w_o);
-  HSA_CHECK_PTR(ctx, o);
-  HSA_CHECK_PTR(ctx, idx);
-  HSA_CHECK_PTR(ctx, x);
+namespace {
+
+// x[idx[m]] += gate * (o[m] W^T) for a [D, D] projection; gate NULL means 1.
+hsa_status proj_residual(hsa_ctx* ctx, const void* w, const void* o, const int32_t* idx, int n,
+                         float* x, const float* gate, const char* what) {
   const int D = ctx->c.cfg.D;
   hsa::GemmArgs g{};
   g.A = o;
-  g.B = w_o;
+  g.B = w;
   g.M = n;
   g.Ncols = D;
   g.Kd = D;
   g.epi = hsa::EPI_RESID;
   g.x = x;
   g.ld_x = D;
+  g.gate = gate;
   g.idx = idx;
   g.N = ctx->c.cfg.N;
   std::string why;
-  return launched(ctx, hsa::launch_gemm(ctx->c, g, &why), "out_proj", why);
+  return launched(ctx, hsa::launch_gemm(ctx->c, g, &why), what, why);
 }
 
-hsa_status hsa_mlp_residual(hsa_ctx* ctx, const void* w_1, const void* w_2, float* x,
-                            const int32_t* idx, int n) {
-  HSA_CHECK_CTX(ctx);
-  if (hsa_status st = check_n(ctx, n)) return st;
-  if (n == 0) return HSA_OK;
-  HSA_CHECK_PTR(ctx, w_1);
-  HSA_CHECK_PTR(ctx, w_2);
-  HSA_CHECK_PTR(ctx, x);
-  HSA_CHECK_PTR(ctx, idx);
+// x[idx[m]] += gate * GELU(u W_1^T) W_2^T with u = LN(x[idx[m]]) * (1 + scale) + shift.
+hsa_status mlp_residual(hsa_ctx* ctx, const void* w_1, const void* w_2, float* x,
+                        const int32_t* idx, int n, const float* shift, const float* scale,
+                        const float* gate) {
   Ctx& c = ctx->c;
   const int D = c.cfg.D, F = c.cfg.F;
-  cudaError_t e = hsa::launch_ln_gather(c, x, idx, n, c.u);
+  cudaError_t e = hsa::launch_ln_gather(c, x, idx, n, c.u, shift, scale);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "ln_gather");
   std::string why;
   hsa::GemmArgs up{};
@@ -420,23 +428,85 @@ hsa_status hsa_mlp_residual(hsa_ctx* ctx, const void* w_1, const void* w_2, floa
   dn.epi = hsa::EPI_RESID;
   dn.x = x;
   dn.ld_x = D;
+  dn.gate = gate;
   dn.idx = idx;
   dn.N = c.cfg.N;
   return launched(ctx, hsa::launch_gemm(c, dn, &why), "mlp_down", why);
 }
 
+}  // namespace
+
+hsa_status hsa_out_proj_residual(hsa_ctx* ctx, const void* w_o, const void* o,
+                                 const int32_t* idx, int n, float* x) {
+  HSA_CHECK_CTX(ctx);
+  if (hsa_status st = check_n(ctx, n)) return st;
+  if (n == 0) return HSA_OK;
+  HSA_CHECK_PTR(ctx, w_o);
+  HSA_CHECK_PTR(ctx, o);
+  HSA_CHECK_PTR(ctx, idx);
+  HSA_CHECK_PTR(ctx, x);
+  return proj_residual(ctx, w_o, o, idx, n, x, nullptr, "out_proj");
+}
+
+
+hsa_status hsa_mlp_residual(hsa_ctx* ctx, const void* w_1, const void* w_2, float* x,
+                            const int32_t* idx, int n) {
+  HSA_CHECK_CTX(ctx);
+  if (hsa_status st = check_n(ctx, n)) return st;
+  if (n == 0) return HSA_OK;
+  HSA_CHECK_PTR(ctx, w_1);
+  HSA_CHECK_PTR(ctx, w_2);
+  HSA_CHECK_PTR(ctx, x);
+  HSA_CHECK_PTR(ctx, idx);
+  return mlp_residual(ctx, w_1, w_2, x, idx, n, nullptr, nullptr, nullptr);
+}
+
 hsa_status hsa_layer_forward(hsa_ctx* ctx, const hsa_layer_weights* w, float* x,
                              const int32_t* idx, int n, void* k_cache, void* v_cache) {
+  return hsa_layer_forward_cond(ctx, w, nullptr, nullptr, x, idx, n, k_cache, v_cache);
+}
+
+hsa_status hsa_layer_forward_cond(hsa_ctx* ctx, const hsa_layer_weights* w, const float* mod,
+                                  const hsa_cross_attn* xa, float* x, const int32_t* idx, int n,
+                                  void* k_cache, void* v_cache) {
   HSA_CHECK_CTX(ctx);
   if (w == nullptr) return fail(ctx, HSA_ERR_INVALID_ARG, "w is NULL");
   if (hsa_status st = check_n(ctx, n)) return st;
+  if (mod != nullptr && (reinterpret_cast<uintptr_t>(mod) & 15) != 0)
+    return fail(ctx, HSA_ERR_INVALID_ARG, "mod must be 16-byte aligned");
+  if (xa != nullptr) {
+    if (xa->n_txt <= 0) return fail(ctx, HSA_ERR_SHAPE, "cross-attention needs n_txt >= 1");
+    if (!xa->w_q || !xa->w_o || !xa->k_txt || !xa->v_txt)
+      return fail(ctx, HSA_ERR_INVALID_ARG, "cross-attention pointer is NULL");
+  }
   if (n == 0) return HSA_OK;
   Ctx& c = ctx->c;
-  hsa_status st = hsa_ln_gather(ctx, x, idx, n, c.u);
-  if (st == HSA_OK) st = hsa_qkv_project(ctx, w->w_qkv, c.u, idx, n, c.q, k_cache, v_cache);
+  const int D = c.cfg.D;
+  // mod rows: shift_a, scale_a, gate_a, shift_m, scale_m, gate_m.
+  const float* m = mod;
+  auto row = [&](int r) { return m == nullptr ? nullptr : m + static_cast<size_t>(r) * D; };
+  HSA_CHECK_PTR(ctx, x);
+  HSA_CHECK_PTR(ctx, idx);
+  cudaError_t e = hsa::launch_ln_gather(c, x, idx, n, c.u, row(0), row(1));
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "ln_gather");
+  hsa_status st = hsa_qkv_project(ctx, w->w_qkv, c.u, idx, n, c.q, k_cache, v_cache);
   if (st == HSA_OK) st = hsa_attention(ctx, c.q, n, k_cache, v_cache, c.o);
-  if (st == HSA_OK) st = hsa_out_proj_residual(ctx, w->w_o, c.o, idx, n, x);
-  if (st == HSA_OK) st = hsa_mlp_residual(ctx, w->w_1, w->w_2, x, idx, n);
+  if (st == HSA_OK) {
+    HSA_CHECK_PTR(ctx, w->w_o);
+    st = proj_residual(ctx, w->w_o, c.o, idx, n, x, row(2), "out_proj");
+  }
+  if (st == HSA_OK && xa != nullptr) {
+    e = hsa::launch_ln_gather(c, x, idx, n, c.u);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "ln_gather");
+    st = hsa_linear(ctx, c.u, n, D, xa->w_q, D, c.q);
+    if (st == HSA_OK) st = hsa_attention_kv(ctx, c.q, n, xa->k_txt, xa->v_txt, xa->n_txt, c.o);
+    if (st == HSA_OK) st = proj_residual(ctx, xa->w_o, c.o, idx, n, x, nullptr, "cross_out_proj");
+  }
+  if (st == HSA_OK) {
+    HSA_CHECK_PTR(ctx, w->w_1);
+    HSA_CHECK_PTR(ctx, w->w_2);
+    st = mlp_residual(ctx, w->w_1, w->w_2, x, idx, n, row(3), row(4), row(5));
+  }
   return st;
 }
 

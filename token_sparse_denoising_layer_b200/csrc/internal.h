@@ -76,7 +76,8 @@ cudaError_t launch_select_groups_raw(cudaStream_t stream, const float* v_prev, c
 cudaError_t launch_selftest_timeout(const Ctx& c, uint64_t limit_ns);
 cudaError_t launch_euler(const Ctx& c, float* x, float* v_hat, float* v_hat_prev,
                          const float* v_fresh, const uint8_t* mask, float s0, float s1);
-cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, int n, void* u);
+cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, int n, void* u,
+                             const float* shift = nullptr, const float* scale = nullptr);
 cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_rows,
                               const int32_t* idx, int n, void* kc, void* vc);
 cudaError_t launch_embed(const Ctx& c, const float* w_in, const float* x_lat, const int32_t* idx,
@@ -103,14 +104,16 @@ struct GemmArgs {
   void* v_cache;      // EPI_QKV
   float* x;           // EPI_RESID
   int ld_x;
+  const float* gate = nullptr;  // EPI_RESID: x[.., j] += gate[j] * C (fp32 [Ncols]) if set
   const int32_t* idx; // EPI_QKV / EPI_RESID
   int N;              // rows of caches / x (bounds for idx)
 };
 
 cudaError_t launch_gemm(const Ctx& c, const GemmArgs& a, std::string* why);
 
+// Attention of n queries against n_kv key/value rows (row stride D).
 cudaError_t launch_attention(const Ctx& c, const void* q, int n, const void* kc, const void* vc,
-                             void* o, std::string* why);
+                             int n_kv, void* o, std::string* why);
 
 // TMA descriptor for a row-major bf16 matrix [rows, cols] with a
 // box of [box_rows, 64] and 128-byte swizzle.  Returns false on failure.

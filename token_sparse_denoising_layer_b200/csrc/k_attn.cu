@@ -396,9 +396,9 @@ __global__ void __launch_bounds__(256) k_attn_combine(AttnParams p) {
 }
 
 template <int HD>
-cudaError_t launch_hd(const Ctx& c, const void* q, int n, const void* kc, const void* vc, void* o,
-                      std::string* why) {
-  const int D = c.cfg.D, N = c.cfg.N;
+cudaError_t launch_hd(const Ctx& c, const void* q, int n, const void* kc, const void* vc, int N,
+                      void* o, std::string* why) {
+  const int D = c.cfg.D;
   CUtensorMap tq, tk, tv;
   if (!make_tmap_bf16(&tq, q, n, D, D, kQ, why)) return cudaErrorInvalidValue;
   if (!make_tmap_bf16(&tk, kc, N, D, D, kKV, why)) return cudaErrorInvalidValue;
@@ -451,11 +451,11 @@ cudaError_t launch_hd(const Ctx& c, const void* q, int n, const void* kc, const 
 }  // namespace
 
 cudaError_t launch_attention(const Ctx& c, const void* q, int n, const void* kc, const void* vc,
-                             void* o, std::string* why) {
+                             int n_kv, void* o, std::string* why) {
   if (n <= 0) return cudaSuccess;
   const int d = c.cfg.D / c.cfg.H;
-  if (d == 128) return launch_hd<128>(c, q, n, kc, vc, o, why);
-  if (d == 64) return launch_hd<64>(c, q, n, kc, vc, o, why);
+  if (d == 128) return launch_hd<128>(c, q, n, kc, vc, n_kv, o, why);
+  if (d == 64) return launch_hd<64>(c, q, n, kc, vc, n_kv, o, why);
   if (why) *why = "attention supports head_dim 64 or 128";
   return cudaErrorInvalidValue;
 }

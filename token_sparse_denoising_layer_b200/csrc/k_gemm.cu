@@ -55,6 +55,7 @@ struct EpiParams {
   __nv_bfloat16* vc;
   float* x;
   int ld_x;
+  const float* gate;
   const int32_t* idx;
   int N;
   int* flag;
@@ -85,16 +86,18 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t
   }
 }
 
-// x[dst .. dst+31] += r (fp32, 128 contiguous bytes).
-__device__ __forceinline__ void add_f32x32(float* dst, const uint32_t (&r)[32]) {
+// x[dst .. dst+31] += r, or += gate[..] * r with a gate (fp32, 128 contiguous bytes).
+__device__ __forceinline__ void add_f32x32(float* dst, const uint32_t (&r)[32], const float* gate) {
   float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
   for (int v = 0; v < 8; ++v) {
     float4 a = d4[v];
-    a.x += __uint_as_float(r[4 * v]);
-    a.y += __uint_as_float(r[4 * v + 1]);
-    a.z += __uint_as_float(r[4 * v + 2]);
-    a.w += __uint_as_float(r[4 * v + 3]);
+    float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
+    if (gate != nullptr) g = __ldg(reinterpret_cast<const float4*>(gate) + v);
+    a.x = fmaf(g.x, __uint_as_float(r[4 * v]), a.x);
+    a.y = fmaf(g.y, __uint_as_float(r[4 * v + 1]), a.y);
+    a.z = fmaf(g.z, __uint_as_float(r[4 * v + 2]), a.z);
+    a.w = fmaf(g.w, __uint_as_float(r[4 * v + 3]), a.w);
     d4[v] = a;
   }
 }
@@ -245,7 +248,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             break;
           }
           case EPI_RESID:
-            if (dst_row >= 0) add_f32x32(p.x + static_cast<size_t>(dst_row) * p.ld_x + col, r);
+            if (dst_row >= 0)
+              add_f32x32(p.x + static_cast<size_t>(dst_row) * p.ld_x + col, r,
+                         p.gate != nullptr ? p.gate + col : nullptr);
             break;
           default:
             break;
@@ -420,7 +425,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
             break;
           }
           case EPI_RESID:
-            if (dst_row >= 0) add_f32x32(p.x + static_cast<size_t>(dst_row) * p.ld_x + col, r);
+            if (dst_row >= 0)
+              add_f32x32(p.x + static_cast<size_t>(dst_row) * p.ld_x + col, r,
+                         p.gate != nullptr ? p.gate + col : nullptr);
             break;
           default:
             break;
@@ -455,6 +462,7 @@ cudaError_t launch_pair(const Ctx& c, const GemmArgs& a, std::string* why) {
   p.vc = static_cast<__nv_bfloat16*>(a.v_cache);
   p.x = a.x;
   p.ld_x = a.ld_x;
+  p.gate = a.gate;
   p.idx = a.idx;
   p.N = a.N;
   p.flag = c.flag;
@@ -487,6 +495,7 @@ cudaError_t launch_bn(const Ctx& c, const GemmArgs& a, std::string* why) {
   p.vc = static_cast<__nv_bfloat16*>(a.v_cache);
   p.x = a.x;
   p.ld_x = a.ld_x;
+  p.gate = a.gate;
   p.idx = a.idx;
   p.N = a.N;
   p.flag = c.flag;

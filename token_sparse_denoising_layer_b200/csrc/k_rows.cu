@@ -44,10 +44,14 @@ __device__ __forceinline__ void row_stats(const float4 (&v)[NCH], int D, float& 
 
 // ------------------------------------------------------------ LN gather
 // One warp per active row: u[m] = bf16(LN(x[idx[m]])).  D = 128 * NCH.
+// With `shift`/`scale` (fp32 [D], both or neither) the normalised row is
+// modulated: u = LN(x) * (1 + scale) + shift.
 template <int NCH>
 __global__ void __launch_bounds__(256) k_ln_gather(const float* __restrict__ x,
                                                    const int32_t* __restrict__ idx, int n, int N,
-                                                   __nv_bfloat16* __restrict__ u, int* flag) {
+                                                   __nv_bfloat16* __restrict__ u, int* flag,
+                                                   const float* __restrict__ shift,
+                                                   const float* __restrict__ scale) {
   const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (m >= n) return;
@@ -67,9 +71,15 @@ __global__ void __launch_bounds__(256) k_ln_gather(const float* __restrict__ x,
   row_stats<NCH>(v, D, mean, rstd);
 #pragma unroll
   for (int c = 0; c < NCH; ++c) {
-    const uint32_t lo = pack_bf16((v[c].x - mean) * rstd, (v[c].y - mean) * rstd);
-    const uint32_t hi = pack_bf16((v[c].z - mean) * rstd, (v[c].w - mean) * rstd);
-    out[c * 32 + lane] = make_uint2(lo, hi);
+    float4 y = make_float4((v[c].x - mean) * rstd, (v[c].y - mean) * rstd,
+                           (v[c].z - mean) * rstd, (v[c].w - mean) * rstd);
+    if (scale != nullptr) {
+      const float4 sc = __ldg(reinterpret_cast<const float4*>(scale) + c * 32 + lane);
+      const float4 sh = __ldg(reinterpret_cast<const float4*>(shift) + c * 32 + lane);
+      y = make_float4(fmaf(y.x, 1.f + sc.x, sh.x), fmaf(y.y, 1.f + sc.y, sh.y),
+                      fmaf(y.z, 1.f + sc.z, sh.z), fmaf(y.w, 1.f + sc.w, sh.w));
+    }
+    out[c * 32 + lane] = make_uint2(pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
   }
 }
 
@@ -77,7 +87,9 @@ __global__ void __launch_bounds__(256) k_ln_gather(const float* __restrict__ x,
 __global__ void __launch_bounds__(256) k_ln_gather_any(const float* __restrict__ x,
                                                        const int32_t* __restrict__ idx, int n,
                                                        int N, int D,
-                                                       __nv_bfloat16* __restrict__ u, int* flag) {
+                                                       __nv_bfloat16* __restrict__ u, int* flag,
+                                                       const float* __restrict__ shift,
+                                                       const float* __restrict__ scale) {
   const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (m >= n) return;
@@ -104,24 +116,32 @@ __global__ void __launch_bounds__(256) k_ln_gather_any(const float* __restrict__
   const float rstd = 1.0f / sqrtf(warp_sum(q) / static_cast<float>(D) + kLnEps);
   for (int c = lane; c < nv; c += 32) {
     const float4 a = __ldg(xr + c);
-    out[c] = make_uint2(pack_bf16((a.x - mean) * rstd, (a.y - mean) * rstd),
-                        pack_bf16((a.z - mean) * rstd, (a.w - mean) * rstd));
+    float4 y = make_float4((a.x - mean) * rstd, (a.y - mean) * rstd, (a.z - mean) * rstd,
+                           (a.w - mean) * rstd);
+    if (scale != nullptr) {
+      const float4 sc = __ldg(reinterpret_cast<const float4*>(scale) + c);
+      const float4 sh = __ldg(reinterpret_cast<const float4*>(shift) + c);
+      y = make_float4(fmaf(y.x, 1.f + sc.x, sh.x), fmaf(y.y, 1.f + sc.y, sh.y),
+                      fmaf(y.z, 1.f + sc.z, sh.z), fmaf(y.w, 1.f + sc.w, sh.w));
+    }
+    out[c] = make_uint2(pack_bf16(y.x, y.y), pack_bf16(y.z, y.w));
   }
 }
 
-cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, int n, void* u) {
+cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, int n, void* u,
+                             const float* shift, const float* scale) {
   if (n <= 0) return cudaSuccess;
   const int D = c.cfg.D, N = c.cfg.N;
   const dim3 grid((n + 7) / 8), block(256);
   auto* uo = static_cast<__nv_bfloat16*>(u);
   switch (D / 128) {
-    case 1: k_ln_gather<1><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
-    case 2: k_ln_gather<2><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
-    case 4: k_ln_gather<4><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
-    case 8: k_ln_gather<8><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
-    case 12: k_ln_gather<12><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
-    case 16: k_ln_gather<16><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag); break;
-    default: k_ln_gather_any<<<grid, block, 0, c.stream>>>(x, idx, n, N, D, uo, c.flag); break;
+    case 1: k_ln_gather<1><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag, shift, scale); break;
+    case 2: k_ln_gather<2><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag, shift, scale); break;
+    case 4: k_ln_gather<4><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag, shift, scale); break;
+    case 8: k_ln_gather<8><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag, shift, scale); break;
+    case 12: k_ln_gather<12><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag, shift, scale); break;
+    case 16: k_ln_gather<16><<<grid, block, 0, c.stream>>>(x, idx, n, N, uo, c.flag, shift, scale); break;
+    default: k_ln_gather_any<<<grid, block, 0, c.stream>>>(x, idx, n, N, D, uo, c.flag, shift, scale); break;
   }
   c.launches += 1;
   return cudaGetLastError();
