@@ -377,6 +377,79 @@ def conditioned_layer(torch, abi):
             "extra_tflops": round(extra_flop / max(cond - plain, 1e-6) / 1e9, 1)}
 
 
+def dit40_steps(torch, synth):
+    """The 40-layer DiT (N = 75600, D = 5120, 40 x 128 heads, F = 13824), budgets
+    {40, 10} at 25/75%: one step at each of its two active patterns (i = 0: all
+    tokens; i = 1: the 25% full-budget group), median of 3 after one warm-up,
+    extrapolated to the 40-step loop (10 all-active steps + 30 at 25%)."""
+    spec = synth.WORKLOADS["dit40_5120"]
+    loop, x0, g0, counts, layers = build_loop(spec, 2, torch)
+    loop.reset(x0, g0)
+    per = {}
+    for i in (0, 1):
+        loop.step(i, False)
+        ts = time_steps_at(loop, i, 3, torch)
+        per[i] = float(np.median(ts))
+    a = {i: loop.n_active(i) for i in (0, 1)}
+    from token_sparse_denoising_layer_b200 import abi
+    abi.hsa_sync_check(loop.ctx)
+    loop.close()
+    del loop, layers
+    torch.cuda.empty_cache()
+    n_full = sum(1 for i in range(spec["T"]) if i % 4 == 0)
+    hsa_loop = n_full * per[0] + (spec["T"] - n_full) * per[1]
+    return {"N": 75600, "D": 5120, "L": 40, "active_i0": a[0], "active_i1": a[1],
+            "ms_step_100%": round(per[0], 1), "ms_step_25%": round(per[1], 1),
+            "hsa_loop_s": round(hsa_loop / 1e3, 2), "dense_loop_s": round(spec["T"] * per[0] / 1e3, 2),
+            "hsa_vs_dense": round(hsa_loop / (spec["T"] * per[0]), 3),
+            "mean_active_fraction": 0.4375}
+
+
+def time_steps_at(loop, i, reps, torch):
+    """CUDA-event times (ms) of `reps` calls of step i (no re-grouping)."""
+    stream = torch.cuda.current_stream()
+    out = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        e0.record(stream)
+        loop.step(i, False)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out.append(e0.elapsed_time(e1))
+    return out
+
+
+def preset_sweep(torch, synth, spec, layers, w_in, w_head, x0_seed=0):
+    """Budget presets and the static split on the 30-layer DiT: the whole 40-step
+    loop per preset (ms per step, mean over the loop).  The pages evaluate four
+    presets and four grouping strategies without defining them; these presets
+    span mean active fractions from 0.75 to 0.44, and "static" keeps the initial
+    seeded random split (no re-grouping) of the default preset."""
+    from token_sparse_denoising_layer_b200.loop import HsaLoop
+    sh = spec["shape"]
+    presets = [("{40,20} 50/50", (40, 20), (0.5, 0.5), True),
+               ("{40,20,10} 40/30/30", (40, 20, 10), (0.4, 0.3, 0.3), True),
+               ("{40,20,10} 40/30/30 static", (40, 20, 10), (0.4, 0.3, 0.3), False),
+               ("{40,10} 25/75", (40, 10), (0.25, 0.75), True),
+               ("{40,20,10,5} 25/25/25/25", (40, 20, 10, 5), (0.25, 0.25, 0.25, 0.25), True)]
+    out = {}
+    for name, budgets, fr, regroup in presets:
+        counts = synth.group_counts(sh.N, fr)
+        loop = HsaLoop(sh.N, sh.D, sh.H, sh.F, layers, w_in, w_head, spec["T"], budgets, counts,
+                       shift=spec["shift"])
+        loop.reset(torch.from_numpy(synth.latent(sh.N, 16, x0_seed)).cuda(),
+                   torch.from_numpy(synth.random_split(sh.N, counts, x0_seed)).cuda())
+        ts = time_steps(loop, spec["T"], torch, regroup=regroup)
+        mean_frac = sum(c * b for c, b in zip(counts, budgets)) / (sh.N * spec["T"])
+        out[name] = {"ms_per_step": round(float(np.mean(ts)), 2),
+                     "mean_active_fraction": round(mean_frac, 4)}
+        loop.close()
+        del loop
+    torch.cuda.empty_cache()
+    return out
+
+
 def cpu_baseline(spec, n_rows=64, target_s=12.0):
     """The oracle on the host cores, on a bounded sample: one layer of the
     30-layer DiT for `n_rows` active rows against the full N = 32760 cache,
@@ -481,6 +554,9 @@ def run_ours(args, rank, world, local, pg):
         sub["euler"] = euler_bandwidth(torch, abi)
         sub["bandwidth"] = bandwidth_sweep(torch, abi)
         sub["conditioned_layer"] = conditioned_layer(torch, abi)
+        sub["presets_dit30"] = preset_sweep(torch, synth, spec, layers, loop.model._keep[0],
+                                            loop.model._keep[1])
+        sub["dit40"] = dit40_steps(torch, synth)
 
     result = None
     if rank == 0:
