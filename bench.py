@@ -46,6 +46,10 @@ def parse():
     ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--mode", choices=["replicas", "shard"], default="replicas",
+                    help="replicas: one loop per GPU (weak scaling); shard: one loop split "
+                         "over the GPUs by active-list chunks with a K/V all-gather per layer "
+                         "(strong scaling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the sub-benchmarks (profiling runs)")
     ap.add_argument("--profile-case", choices=["attention", "gemm", "euler"], default=None,
@@ -614,6 +618,97 @@ def run_ours(args, rank, world, local, pg):
     return result
 
 
+def run_shard(args, rank, world, local, pg):
+    """One 30-layer DiT loop split over the ranks (sequence-sharded step):
+    every rank runs its chunk of each step's active list; ms per step is the
+    max over ranks of the device-timed region."""
+    import torch
+
+    from token_sparse_denoising_layer_b200 import abi, synth
+    from token_sparse_denoising_layer_b200.shard import ShardRank, run_dist, run_local
+
+    torch.cuda.set_device(local)
+    spec = synth.WORKLOADS[WORKLOAD]
+    sh = spec["shape"]
+    counts = synth.group_counts(sh.N, spec["fractions"])
+    # the same seed on every rank: one model, one latent, one initial split
+    layers = [synth.device_layer_weights(sh.D, sh.F, l) for l in range(sh.L)]
+    wf = synth.model_weights(synth.ModelShape(sh.N, sh.C, sh.D, sh.H, 64, 0), 0)
+    rk = ShardRank(rank, world, sh.N, sh.D, sh.H, sh.F, layers,
+                   torch.from_numpy(wf["w_in"]).cuda(), torch.from_numpy(wf["w_head"]).cuda(),
+                   spec["T"], spec["budgets"], counts, shift=spec["shift"])
+    x0 = torch.from_numpy(synth.latent(sh.N, 16, 0)).cuda()
+    g0 = torch.from_numpy(synth.random_split(sh.N, counts, 0)).cuda()
+
+    def step(i):
+        if pg is not None:
+            run_dist(rk.steps(i, True))
+        else:
+            run_local([rk.steps(i, True)])
+
+    def timed(k_steps, hook=None):
+        stream = torch.cuda.current_stream()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+              for _ in range(k_steps)]
+        torch.cuda.synchronize()
+        for k in range(k_steps):
+            ev[k][0].record(stream)
+            (hook or (lambda kk, ii: step(ii)))(k, k % spec["T"])
+            ev[k][1].record(stream)
+        torch.cuda.synchronize()
+        return [a.elapsed_time(b) for a, b in ev]
+
+    rk.reset(x0, g0)
+    for k in range(args.warmup):
+        step(k % spec["T"])
+    abi.hsa_sync_check(rk.ctx)
+    rk.reset(x0, g0)
+    barrier(pg)
+    launches0 = abi.hsa_kernel_launches(rk.ctx)
+    with ClockSampler(local) as clk:
+        times = timed(args.steps)
+    launches = abi.hsa_kernel_launches(rk.ctx) - launches0
+    abi.hsa_sync_check(rk.ctx)
+    dev = torch.device("cuda", local)
+    ms_step = max_over_ranks(float(np.sum(times)), pg, dev) / args.steps
+    barrier(pg)
+    x_host = [torch.empty((sh.N, 16), dtype=torch.float32).pin_memory() for _ in range(2)]
+    x_host[0].copy_(x0.cpu())
+    rk.reset(x0, g0)
+
+    def e2e_hook(k, i):
+        rk.x.copy_(x_host[k % 2], non_blocking=True)
+        step(i)
+        x_host[(k + 1) % 2].copy_(rk.x, non_blocking=True)
+
+    e2e_ms = max_over_ranks(float(np.sum(timed(args.steps, e2e_hook))), pg, dev) / args.steps
+    launches_all = max_over_ranks(float(launches), pg, dev) * world
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": round(ms_step, 3), "unit": "ms/step", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 3),
+            "higher_is_better": False, "scaling": "strong", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic (seeded; random N(0,1/fan_in) weights, x ~ N(0,1))",
+            "config": {"workload": "HSA loop, 30-layer DiT: N=32760 (21x30x52), C=16, D=1536, "
+                                   "H=12x128, F=8960, T=40, shift 5, budgets {40,20,10} at "
+                                   "40/30/30%, regroup by L1 relative velocity change",
+                       "global_batch": 1, "seq_len": sh.N,
+                       "parallelism": f"sequence-shard x{world} (active-list chunks, K|V "
+                                      f"all-gather per layer, velocity all-reduce per step)",
+                       "l2": "inputs larger than L2 (>8 GB touched per step)",
+                       "step": "one global iteration i = k mod 40; 40 steps = one loop",
+                       "value": "ms per step of the one loop, max over ranks"},
+            "mean_active_fraction": 0.625,
+            "gpu_launches": int(launches_all),
+            "e2e": {"value": round(e2e_ms, 3), "unit": "ms/step",
+                    "h2d_bytes_per_step": sh.N * 16 * 4, "d2h_bytes_per_step": sh.N * 16 * 4},
+            "clocks": clk.summary(),
+        }
+    rk.close()
+    return result
+
+
 # --------------------------------------------------------------------------- reference arm
 
 def run_reference(args, rank, world):
@@ -711,7 +806,7 @@ def main():
             print(json.dumps(res), flush=True)
         return 0
     rank, world, local, pg = dist_setup(args.gpus)
-    res = run_ours(args, rank, world, local, pg)
+    res = (run_shard if args.mode == "shard" else run_ours)(args, rank, world, local, pg)
     if rank == 0 and res is not None:
         print(json.dumps(res), flush=True)
     if pg is not None:

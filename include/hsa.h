@@ -206,6 +206,17 @@ hsa_status hsa_kv_scatter(hsa_ctx* ctx, const void* k_rows, const void* v_rows,
                           const int32_t* idx, int n, void* k_cache, void* v_cache);
 
 /*
+ * The same KV-cache write from packed rows, as a sequence-sharded step
+ * receives them after gathering every rank's fresh rows ([TS] 2.2 step 2):
+ * k_cache[idx[m]] = kv_rows[m][0 .. D), v_cache[idx[m]] = kv_rows[m][D .. 2D).
+ *   kv_rows (device) bf16 [n, 2D];  idx (device) int32 [n], each < N;
+ *   k_cache, v_cache (device) bf16 [N, D].  An index outside [0, N) is skipped
+ *   and reported by hsa_sync_check (HSA_ERR_DEVICE_CHECK).
+ */
+hsa_status hsa_kv_scatter_packed(hsa_ctx* ctx, const void* kv_rows, const int32_t* idx, int n,
+                                 void* k_cache, void* v_cache);
+
+/*
  * Full-context attention of the active queries ([TS] 2.2 steps 3-4):
  * per head, o[m] = softmax(q[m] K^T / sqrt(d)) V over all N cached rows,
  * fp32 accumulation, online softmax.  Cost O(n * N).

@@ -1,0 +1,153 @@
+"""GPU parity of the sequence-sharded step (one loop split over G ranks).
+
+Ranks are emulated in one process on one GPU (their exchanges are device
+copies between their buffers, and no kernel waits on another rank), and a
+world of one runs through torch.distributed with NCCL.  Every rank must end
+with the same latent bit for bit (the replicated parts are deterministic);
+the result must match the unsharded loop and the float64 oracle.
+"""
+
+import datetime
+import os
+import socket
+
+import numpy as np
+import pytest
+
+from gpu_util import bf, dev, host, need_gpu, torch
+from oracle import hsa_oracle as O
+from token_sparse_denoising_layer_b200 import abi, synth
+
+pytestmark = pytest.mark.gpu
+
+
+def test_kv_scatter_packed_is_an_exact_copy():
+    need_gpu()
+    N, D, a = 700, 256, 333
+    ctx = abi.hsa_create(N=N, D=D, H=2, F=64, L=1, T=1, budgets=[1], counts=[N])
+    ks, vs = synth.stale_kv(N, D, 31)
+    idx = synth.random_active_set(N, a, 31)
+    kv = synth.bf16_round(synth.rng(32).standard_normal((a, 2 * D), dtype=np.float32))
+    kc, vc = bf(ks), bf(vs)
+    abi.hsa_kv_scatter_packed(ctx, bf(kv), dev(idx), a, kc, vc)
+    abi.hsa_sync_check(ctx)
+    want_k, want_v = ks.copy(), vs.copy()
+    want_k[idx] = kv[:, :D]
+    want_v[idx] = kv[:, D:]
+    assert (host(kc) == want_k).all() and (host(vc) == want_v).all()
+    ctx.close()
+
+
+def _model(name, N=None, L=None):
+    spec = synth.WORKLOADS[name]
+    sh = spec["shape"]
+    if N is not None:
+        sh = synth.ModelShape(N=N, C=16, D=sh.D, H=sh.H, F=sh.F, L=L if L is not None else sh.L)
+    counts = synth.group_counts(sh.N, spec["fractions"])
+    w = synth.model_weights(sh, 9)
+    layers = [tuple(bf(lw[k]) for k in ("w_qkv", "w_o", "w_1", "w_2")) for lw in w["layers"]]
+    return spec, sh, counts, w, layers
+
+
+def _run_sharded(G, spec, sh, counts, w, layers, regroup):
+    from token_sparse_denoising_layer_b200.shard import ShardRank, run_local
+
+    ranks = [ShardRank(r, G, sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]),
+                       spec["T"], spec["budgets"], counts, shift=spec["shift"]) for r in range(G)]
+    x0 = synth.latent(sh.N, 16, 9)
+    g0 = synth.random_split(sh.N, counts, 9)
+    for rk in ranks:
+        rk.reset(dev(x0), dev(g0))
+    for i in range(spec["T"]):
+        run_local([rk.steps(i, regroup) for rk in ranks])
+    for rk in ranks:
+        abi.hsa_sync_check(rk.ctx)
+    out = [host(rk.x) for rk in ranks]
+    g = [host(rk.g) for rk in ranks]
+    for rk in ranks:
+        rk.close()
+    return x0, g0, out, g
+
+
+def _run_single(spec, sh, counts, w, layers, x0, g0, regroup):
+    from token_sparse_denoising_layer_b200.loop import HsaLoop
+
+    loop = HsaLoop(sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]), spec["T"],
+                   spec["budgets"], counts, shift=spec["shift"])
+    loop.reset(x0, g0)
+    loop.run(regroup=regroup)
+    abi.hsa_sync_check(loop.ctx)
+    x = host(loop.x)
+    loop.close()
+    return x
+
+
+def _rel(a, b):
+    return float(np.linalg.norm(a - b) / np.linalg.norm(b))
+
+
+@pytest.mark.parametrize("G", [1, 2, 3])
+@pytest.mark.parametrize("regroup", [False, True])
+def test_sharded_tiny_dit_matches_single_gpu_loop(G, regroup):
+    need_gpu()
+    spec, sh, counts, w, layers = _model("tiny_dit")
+    x0, g0, xs, gs = _run_sharded(G, spec, sh, counts, w, layers, regroup)
+    for r in range(1, G):
+        assert np.array_equal(xs[r], xs[0]) and np.array_equal(gs[r], gs[0])
+    x1 = _run_single(spec, sh, counts, w, layers, x0, g0, regroup)
+    d = _rel(xs[0], x1)
+    print(f"G={G} regroup={regroup}: sharded vs single-GPU loop {d:.2e} "
+          f"(bitwise: {np.array_equal(xs[0], x1)})")
+    assert d <= 1e-2
+    xr = O.run_loop(w, x0, g0, spec["T"], list(spec["budgets"]), counts,
+                    O.sigma_schedule(spec["T"], spec["shift"]), sh.H, regroup=regroup)
+    assert _rel(xs[0], xr) <= 2e-2
+
+
+def test_sharded_dit30_shapes_three_ranks():
+    """The 30-layer DiT's D, H, F, T and budgets with one layer and N = 840:
+    several 128-row tiles per rank and ragged chunks (a = 840, 588, 336)."""
+    need_gpu()
+    spec, sh, counts, w, layers = _model("dit30_1536", N=840, L=1)
+    x0, g0, xs, gs = _run_sharded(3, spec, sh, counts, w, layers, True)
+    assert np.array_equal(xs[1], xs[0]) and np.array_equal(xs[2], xs[0])
+    x1 = _run_single(spec, sh, counts, w, layers, x0, g0, True)
+    d = _rel(xs[0], x1)
+    print(f"dit30 shapes, G=3: sharded vs single-GPU loop {d:.2e}")
+    assert d <= 1e-2
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def test_sharded_world_of_one_through_nccl():
+    """run_dist over a real NCCL process group of size 1 equals the in-process
+    driver bit for bit."""
+    need_gpu()
+    import torch.distributed as dist
+
+    from token_sparse_denoising_layer_b200.shard import ShardRank, run_dist
+
+    spec, sh, counts, w, layers = _model("tiny_dit")
+    x0, g0, xs, _ = _run_sharded(1, spec, sh, counts, w, layers, True)
+    store = dist.TCPStore("127.0.0.1", _free_port(), 1, True,
+                          timeout=datetime.timedelta(seconds=60))
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        rk = ShardRank(0, 1, sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]),
+                       spec["T"], spec["budgets"], counts, shift=spec["shift"])
+        rk.reset(dev(x0), dev(g0))
+        for i in range(spec["T"]):
+            run_dist(rk.steps(i, True))
+        abi.hsa_sync_check(rk.ctx)
+        assert np.array_equal(host(rk.x), xs[0])
+        rk.close()
+    finally:
+        dist.destroy_process_group()

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(PKG, "libhsa.so")
 SYMBOLS = [
     "hsa_create", "hsa_destroy", "hsa_last_error", "hsa_set_stream", "hsa_sync_check",
     "hsa_selftest_timeout", "hsa_kernel_launches", "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
-    "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_linear", "hsa_kv_scatter",
+    "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_linear", "hsa_kv_scatter", "hsa_kv_scatter_packed",
     "hsa_attention", "hsa_attention_kv", "hsa_out_proj_residual", "hsa_mlp_residual",
     "hsa_layer_forward", "hsa_layer_forward_cond", "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_step", "hsa_select_groups_static",
 ]
@@ -97,6 +97,7 @@ def load() -> ctypes.CDLL:
         "hsa_qkv_project": (I, [P, P, P, P, I, P, P, P]),
         "hsa_linear": (I, [P, P, I, I, P, I, P]),
         "hsa_kv_scatter": (I, [P, P, P, P, I, P, P]),
+        "hsa_kv_scatter_packed": (I, [P, P, P, I, P, P]),
         "hsa_attention": (I, [P, P, I, P, P, P]),
         "hsa_attention_kv": (I, [P, P, I, P, P, I, P]),
         "hsa_out_proj_residual": (I, [P, P, P, P, I, P]),
@@ -233,6 +234,11 @@ def hsa_linear(ctx: Context, a, M: int, Kd: int, w, Ncols: int, out) -> None:
 def hsa_kv_scatter(ctx: Context, k_rows, v_rows, idx, n: int, k_cache, v_cache) -> None:
     _check(ctx.ptr, load().hsa_kv_scatter(ctx.ptr, _p(k_rows), _p(v_rows), _p(idx), n,
                                           _p(k_cache), _p(v_cache)))
+
+
+def hsa_kv_scatter_packed(ctx: Context, kv_rows, idx, n: int, k_cache, v_cache) -> None:
+    _check(ctx.ptr, load().hsa_kv_scatter_packed(ctx.ptr, _p(kv_rows), _p(idx), n, _p(k_cache),
+                                                 _p(v_cache)))
 
 
 def hsa_attention(ctx: Context, q, n: int, k_cache, v_cache, o) -> None:

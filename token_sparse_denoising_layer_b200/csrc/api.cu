@@ -343,8 +343,26 @@ hsa_status hsa_kv_scatter(hsa_ctx* ctx, const void* k_rows, const void* v_rows,
   HSA_CHECK_PTR(ctx, idx);
   HSA_CHECK_PTR(ctx, k_cache);
   HSA_CHECK_PTR(ctx, v_cache);
-  return launched(ctx, hsa::launch_kv_scatter(ctx->c, k_rows, v_rows, idx, n, k_cache, v_cache),
+  return launched(ctx,
+                  hsa::launch_kv_scatter(ctx->c, k_rows, v_rows, ctx->c.cfg.D, idx, n, k_cache,
+                                         v_cache),
                   "kv_scatter");
+}
+
+hsa_status hsa_kv_scatter_packed(hsa_ctx* ctx, const void* kv_rows, const int32_t* idx, int n,
+                                 void* k_cache, void* v_cache) {
+  HSA_CHECK_CTX(ctx);
+  if (hsa_status st = check_n(ctx, n)) return st;
+  if (n == 0) return HSA_OK;
+  HSA_CHECK_PTR(ctx, kv_rows);
+  HSA_CHECK_PTR(ctx, idx);
+  HSA_CHECK_PTR(ctx, k_cache);
+  HSA_CHECK_PTR(ctx, v_cache);
+  const int D = ctx->c.cfg.D;
+  const void* v_rows = static_cast<const uint16_t*>(kv_rows) + D;
+  return launched(ctx,
+                  hsa::launch_kv_scatter(ctx->c, kv_rows, v_rows, 2 * D, idx, n, k_cache, v_cache),
+                  "kv_scatter_packed");
 }
 
 hsa_status hsa_attention(hsa_ctx* ctx, const void* q, int n, const void* k_cache,

@@ -78,7 +78,7 @@ cudaError_t launch_euler(const Ctx& c, float* x, float* v_hat, float* v_hat_prev
                          const float* v_fresh, const uint8_t* mask, float s0, float s1);
 cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, int n, void* u,
                              const float* shift = nullptr, const float* scale = nullptr);
-cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_rows,
+cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_rows, int src_ld,
                               const int32_t* idx, int n, void* kc, void* vc);
 cudaError_t launch_embed(const Ctx& c, const float* w_in, const float* x_lat, const int32_t* idx,
                          int n, float* h);

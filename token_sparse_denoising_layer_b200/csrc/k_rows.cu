@@ -149,8 +149,9 @@ cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, i
 
 // ------------------------------------------------------------ KV scatter
 // k_cache[idx[m]] = k_rows[m], v_cache[idx[m]] = v_rows[m]; 16-byte vectors.
+// Source row m of K (V) starts at k_rows (v_rows) + m * src_ld, in 16-byte units.
 __global__ void __launch_bounds__(256) k_kv_scatter(const uint4* __restrict__ k_rows,
-                                                    const uint4* __restrict__ v_rows,
+                                                    const uint4* __restrict__ v_rows, int src_ld,
                                                     const int32_t* __restrict__ idx, int n, int N,
                                                     int vec_per_row, uint4* __restrict__ kc,
                                                     uint4* __restrict__ vc, int* flag) {
@@ -162,12 +163,13 @@ __global__ void __launch_bounds__(256) k_kv_scatter(const uint4* __restrict__ k_
     const int r = __ldg(idx + m);
     if (!row_ok(r, N, flag)) continue;
     const size_t dst = static_cast<size_t>(r) * vec_per_row + c;
-    __stcs(kc + dst, __ldcs(k_rows + t));
-    __stcs(vc + dst, __ldcs(v_rows + t));
+    const size_t src = static_cast<size_t>(m) * src_ld + c;
+    __stcs(kc + dst, __ldcs(k_rows + src));
+    __stcs(vc + dst, __ldcs(v_rows + src));
   }
 }
 
-cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_rows,
+cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_rows, int src_ld,
                               const int32_t* idx, int n, void* kc, void* vc) {
   if (n <= 0) return cudaSuccess;
   const int vpr = c.cfg.D / 8;
@@ -176,7 +178,8 @@ cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_ro
   const size_t cap = static_cast<size_t>(c.num_sms) * 16;
   if (blocks > cap) blocks = cap;
   k_kv_scatter<<<static_cast<unsigned>(blocks), 256, 0, c.stream>>>(
-      static_cast<const uint4*>(k_rows), static_cast<const uint4*>(v_rows), idx, n, c.cfg.N, vpr,
+      static_cast<const uint4*>(k_rows), static_cast<const uint4*>(v_rows), src_ld / 8, idx, n,
+      c.cfg.N, vpr,
       static_cast<uint4*>(kc), static_cast<uint4*>(vc), c.flag);
   c.launches += 1;
   return cudaGetLastError();

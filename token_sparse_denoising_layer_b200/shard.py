@@ -1,0 +1,208 @@
+"""Sequence-sharded HSA step: one loop split over G ranks (one GPU each).
+
+"Technical Summary: Heterogeneous Step Allocation (HSA) for Efficient Video
+Generation", section 2.2: every active token writes fresh K/V rows into the
+per-layer cache, then every active query attends to all N cached rows.  So
+the active list A_i of a step splits across ranks with one exchange per
+layer: each rank runs QKV, attention, out-projection and MLP for its share of
+A_i, and the fresh K/V rows of all shares are gathered into every rank's copy
+of the cache before attention reads it.
+
+Partition.  A_i (ascending, identical on every rank because the group ids
+are) is cut into G chunks of c positions, c = ceil(a / G) rounded up to a
+multiple of 4 so that every chunk of the int32 list starts on a 16-byte
+boundary; rank r takes positions [r c, min(a, (r+1) c)).  Only trailing
+chunks can be short, so after an all-gather of c-row chunks the first a rows,
+in rank order, are the fresh rows of A_i in order and scatter straight into
+the cache by A_i.
+
+Per step on rank r:
+  schedule (all of A_i) -> embed, L x [LN, Q and K|V GEMMs of its chunk,
+  all-gather K|V, scatter into the cache, attention of its queries against
+  all N rows, out-projection + MLP] -> head of its chunk into a zeroed [N, C]
+  buffer -> all-reduce (sum) of that buffer, which is exact because every
+  active row has exactly one non-zero contributor -> cached Euler over all N
+  (replicated) -> re-grouping (replicated; deterministic, so the group ids
+  stay identical on every rank).
+
+Every step of the path runs in libhsa's kernels; the exchanges are
+collectives.  The step is written once, as a generator that yields each
+exchange; `run_dist` serves the requests with torch.distributed (NCCL on
+GPUs, gloo in CPU tests) and `run_local` serves G ranks held in one process
+by copying between their buffers.
+"""
+
+from __future__ import annotations
+
+from typing import Iterator, List, Sequence, Tuple
+
+from . import abi
+from .loop import sigma_schedule
+
+
+CHUNK_ALIGN = 4  # int32 entries per 16 bytes
+
+
+def chunk_rows(a: int, G: int) -> int:
+    """Rows per rank for a active tokens: ceil(a / G), rounded up to CHUNK_ALIGN."""
+    c = -(-a // G)
+    return max(CHUNK_ALIGN, -(-c // CHUNK_ALIGN) * CHUNK_ALIGN)
+
+
+def shard_slices(a: int, G: int) -> Tuple[int, List[Tuple[int, int]]]:
+    """Chunk size c and each rank's (start, count) within the active list."""
+    if G < 1 or a < 0:
+        raise ValueError("need G >= 1 and a >= 0")
+    c = chunk_rows(a, G)
+    out = []
+    for r in range(G):
+        s = min(a, r * c)
+        out.append((s, min(a, s + c) - s))
+    return c, out
+
+
+Request = Tuple  # ("all_gather", send, recv) | ("all_reduce_sum", buf)
+
+
+class ShardRank:
+    """One rank's device state for the sharded loop.
+
+    The latent, velocity caches, group ids and the per-layer K/V caches are
+    replicated ([N, ...] on every rank); the hidden rows h are [N, D] but a
+    rank only touches the rows of its chunk.  ``layers`` holds the bf16 CUDA
+    tensors (w_qkv, w_o, w_1, w_2) per block; w_in [D, C] and w_head [C, D]
+    are float32.
+    """
+
+    def __init__(self, rank: int, G: int, N: int, D: int, H: int, F: int, layers, w_in, w_head,
+                 T: int, budgets: Sequence[int], counts: Sequence[int], shift: float = 1.0,
+                 m: int = 0, stream=None):
+        import torch
+
+        if not 0 <= rank < G:
+            raise ValueError("rank outside [0, G)")
+        self.torch = torch
+        self.rank, self.G = rank, G
+        self.N, self.D, self.H, self.F, self.L = N, D, H, F, len(layers)
+        self.T, self.budgets, self.counts = T, list(budgets), list(counts)
+        self.ctx = abi.hsa_create(N=N, D=D, H=H, F=F, L=self.L, T=T, budgets=budgets,
+                                  counts=counts, m=m, stream=stream)
+        f32 = dict(dtype=torch.float32, device="cuda")
+        bf = dict(dtype=torch.bfloat16, device="cuda")
+        self.x = torch.zeros((N, 16), **f32)
+        self.v_hat = torch.zeros((N, 16), **f32)
+        self.v_hat_prev = torch.zeros((N, 16), **f32)
+        self.v_stage = torch.zeros((N, 16), **f32)
+        self.score = torch.zeros((N,), **f32)
+        self.g = torch.zeros((N,), dtype=torch.uint8, device="cuda")
+        self.mask = torch.zeros((N,), dtype=torch.uint8, device="cuda")
+        self.active_idx = torch.zeros((N,), dtype=torch.int32, device="cuda")
+        self.h = torch.zeros((N, D), **f32)
+        self.k_cache = [torch.zeros((N, D), **bf) for _ in layers]
+        self.v_cache = [torch.zeros((N, D), **bf) for _ in layers]
+        cmax = chunk_rows(N, G)
+        self.u = torch.empty((cmax, D), **bf)
+        self.q = torch.empty((cmax, D), **bf)
+        self.o = torch.empty((cmax, D), **bf)
+        self.kv_send = torch.empty((cmax, 2 * D), **bf)
+        self.kv_recv = torch.empty((G * cmax, 2 * D), **bf)
+        # W_qkv rows [0, D) project Q, rows [D, 3D) project K|V: contiguous views
+        self.w_q = [lw[0][:D] for lw in layers]
+        self.w_kv = [lw[0][D:] for lw in layers]
+        self.layers = layers
+        self.w_in, self.w_head = w_in, w_head
+        self.sigmas = sigma_schedule(T, shift)
+
+    def reset(self, x0, g0) -> None:
+        """Start a run from latent x0 [N, 16] and group ids g0 [N] (same on every rank)."""
+        t = self.torch
+        self.x.copy_(t.as_tensor(x0))
+        self.g.copy_(t.as_tensor(g0))
+        for buf in (self.v_hat, self.v_hat_prev, self.v_stage, self.score):
+            buf.zero_()
+
+    def steps(self, i: int, regroup: bool = True) -> Iterator[Request]:
+        """Global iteration i on this rank; yields at each exchange."""
+        ctx, D = self.ctx, self.D
+        a = abi.hsa_schedule(ctx, i, self.g, self.mask, self.active_idx)
+        c, sl = shard_slices(a, self.G)
+        s0, nr = sl[self.rank]
+        idx_r = self.active_idx[s0:s0 + nr]
+        abi.hsa_embed(ctx, self.w_in, self.x, idx_r, nr, self.h)
+        for l in range(self.L):
+            _, w_o, w_1, w_2 = self.layers[l]
+            abi.hsa_ln_gather(ctx, self.h, idx_r, nr, self.u)
+            abi.hsa_linear(ctx, self.u, nr, D, self.w_q[l], D, self.q)
+            abi.hsa_linear(ctx, self.u, nr, D, self.w_kv[l], 2 * D, self.kv_send)
+            yield ("all_gather", self.kv_send[:c], self.kv_recv[:self.G * c])
+            abi.hsa_kv_scatter_packed(ctx, self.kv_recv, self.active_idx, a, self.k_cache[l],
+                                      self.v_cache[l])
+            abi.hsa_attention(ctx, self.q, nr, self.k_cache[l], self.v_cache[l], self.o)
+            abi.hsa_out_proj_residual(ctx, w_o, self.o, idx_r, nr, self.h)
+            abi.hsa_mlp_residual(ctx, w_1, w_2, self.h, idx_r, nr)
+        self.v_stage.zero_()
+        abi.hsa_head(ctx, self.w_head, self.h, idx_r, nr, self.v_stage)
+        yield ("all_reduce_sum", self.v_stage)
+        abi.hsa_euler_step(ctx, self.x, self.v_hat, self.v_hat_prev, self.v_stage, self.mask,
+                           float(self.sigmas[i]), float(self.sigmas[i + 1]))
+        if regroup and self.T // self.budgets[-1] <= i < self.T - 1:
+            abi.hsa_select_groups(ctx, self.v_hat_prev, self.v_hat, self.score, self.g)
+
+    def n_active(self, i: int) -> int:
+        return abi.hsa_n_active(self.ctx, i)
+
+    def close(self) -> None:
+        self.ctx.close()
+
+
+def _serve_dist(req: Request, group) -> None:
+    import torch.distributed as dist
+
+    if req[0] == "all_gather":
+        _, send, recv = req
+        if dist.get_backend(group) == "nccl":
+            dist.all_gather_into_tensor(recv, send, group=group)
+        else:
+            dist.all_gather(list(recv.chunk(dist.get_world_size(group))), send, group=group)
+    elif req[0] == "all_reduce_sum":
+        dist.all_reduce(req[1], op=dist.ReduceOp.SUM, group=group)
+    else:
+        raise ValueError(f"unknown exchange {req[0]!r}")
+
+
+def run_dist(steps: Iterator[Request], group=None) -> None:
+    """Drive one rank's step generator with torch.distributed collectives.
+
+    Every rank yields the same requests in the same order (the same number of
+    layers, one reduction per step), so the collectives match across ranks."""
+    for req in steps:
+        _serve_dist(req, group)
+
+
+def run_local(all_steps: Sequence[Iterator[Request]]) -> None:
+    """Drive G ranks held in one process in lockstep, exchanging by copies."""
+    gens = list(all_steps)
+    while True:
+        reqs = []
+        for g in gens:
+            try:
+                reqs.append(next(g))
+            except StopIteration:
+                reqs.append(None)
+        if all(r is None for r in reqs):
+            return
+        if any(r is None for r in reqs) or len({r[0] for r in reqs}) != 1:
+            raise RuntimeError("ranks diverged: different exchange requests")
+        op = reqs[0][0]
+        if op == "all_gather":
+            for _, _, recv in reqs:
+                for r, (_, send, _) in enumerate(reqs):
+                    recv[r * send.shape[0]:(r + 1) * send.shape[0]].copy_(send)
+        elif op == "all_reduce_sum":
+            total = reqs[0][1].clone()
+            for r in reqs[1:]:
+                total += r[1]
+            for r in reqs:
+                r[1].copy_(total)
+        else:
+            raise ValueError(f"unknown exchange {op!r}")
