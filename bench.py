@@ -454,6 +454,59 @@ def preset_sweep(torch, synth, spec, layers, w_in, w_head, x0_seed=0):
     return out
 
 
+def graph_replay(torch, synth, loop, x0, g0, eager_ms):
+    """The loop recorded as one CUDA graph (40 steps, one launch from the host)
+    against eager launches: the tiny DiT (N = 256, launch-bound) and the
+    30-layer DiT (the bench loop itself)."""
+    from token_sparse_denoising_layer_b200.loop import HsaLoop
+
+    def time_replay(lp, reps):
+        stream = torch.cuda.current_stream()
+        out = []
+        for _ in range(reps):
+            lp.reset(x0_of[id(lp)], g0_of[id(lp)])
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            e0.record(stream)
+            lp.replay()
+            e1.record(stream)
+            torch.cuda.synchronize()
+            out.append(e0.elapsed_time(e1) / lp.T)
+        return float(np.median(out))
+
+    spec = synth.WORKLOADS["tiny_dit"]
+    sh = spec["shape"]
+    counts = synth.group_counts(sh.N, spec["fractions"])
+    w = synth.model_weights(sh, 0)
+    layers = [tuple(torch.from_numpy(lw[k]).to(torch.bfloat16).cuda()
+                    for k in ("w_qkv", "w_o", "w_1", "w_2")) for lw in w["layers"]]
+    tiny = HsaLoop(sh.N, sh.D, sh.H, sh.F, layers, torch.from_numpy(w["w_in"]).cuda(),
+                   torch.from_numpy(w["w_head"]).cuda(), spec["T"], spec["budgets"], counts,
+                   shift=spec["shift"])
+    tx0 = torch.from_numpy(synth.latent(sh.N, 16, 0)).cuda()
+    tg0 = torch.from_numpy(synth.random_split(sh.N, counts, 0)).cuda()
+    x0_of = {id(tiny): tx0, id(loop): x0}
+    g0_of = {id(tiny): tg0, id(loop): g0}
+    tiny.reset(tx0, tg0)
+    tiny.run()
+    tiny.reset(tx0, tg0)
+    tiny_eager = float(np.median(time_steps(tiny, 5 * spec["T"], torch)))
+    tiny.capture()
+    tiny_graph = time_replay(tiny, 5)
+    loop.reset(x0, g0)
+    loop.capture()
+    big_graph = time_replay(loop, 2)
+    out = {"tiny_dit": {"eager_ms_per_step": round(tiny_eager, 4),
+                        "graph_ms_per_step": round(tiny_graph, 4),
+                        "launches_per_loop": tiny.graph_launches},
+           "dit30_1536": {"eager_ms_per_step": round(eager_ms, 3),
+                          "graph_ms_per_step": round(big_graph, 3),
+                          "launches_per_loop": loop.graph_launches}}
+    tiny.close()
+    loop.graph = None
+    return out
+
+
 def cpu_baseline(spec, n_rows=64, target_s=12.0):
     """The oracle on the host cores, on a bounded sample: one layer of the
     30-layer DiT for `n_rows` active rows against the full N = 32760 cache,
@@ -561,6 +614,7 @@ def run_ours(args, rank, world, local, pg):
         sub["presets_dit30"] = preset_sweep(torch, synth, spec, layers, loop.model._keep[0],
                                             loop.model._keep[1])
         sub["dit40"] = dit40_steps(torch, synth)
+        sub["cuda_graph"] = graph_replay(torch, synth, loop, x0, g0, ms_step)
 
     result = None
     if rank == 0:

@@ -40,6 +40,9 @@ class HsaLoop:
         self.T, self.budgets, self.counts = T, list(budgets), list(counts)
         self.ctx = abi.hsa_create(N=N, D=D, H=H, F=F, L=self.L, T=T, budgets=budgets,
                                   counts=counts, m=m, stream=stream)
+        self._stream = stream
+        self.graph = None
+        self.graph_launches = 0
         dev = "cuda"
         f32 = dict(dtype=torch.float32, device=dev)
         self.x = torch.zeros((N, 16), **f32)
@@ -78,5 +81,34 @@ class HsaLoop:
             self.step(i, regroup)
         return self.x
 
+    def capture(self, regroup: bool = True) -> None:
+        """Record the whole loop, i = 0..T-1, as one CUDA graph.
+
+        Every step's launch shape is fixed by the host (|A_i| follows from the
+        group counts), so the T steps replay as recorded; the graph reads and
+        writes this loop's buffers in place.  Call after at least one eager
+        step (first calls set kernel attributes), and reset() before replay()."""
+        t = self.torch
+        t.cuda.synchronize()
+        side = t.cuda.Stream()
+        g = t.cuda.CUDAGraph()
+        n0 = abi.hsa_kernel_launches(self.ctx)
+        abi.hsa_set_stream(self.ctx, side)
+        try:
+            with t.cuda.graph(g, stream=side):
+                for i in range(self.T):
+                    self.step(i, regroup)
+        finally:
+            abi.hsa_set_stream(self.ctx, self._stream)
+        self.graph_launches = abi.hsa_kernel_launches(self.ctx) - n0
+        self.graph = g
+
+    def replay(self) -> None:
+        """Run the recorded loop on the current stream."""
+        if self.graph is None:
+            raise RuntimeError("capture() first")
+        self.graph.replay()
+
     def close(self) -> None:
+        self.graph = None
         self.ctx.close()
