@@ -258,6 +258,69 @@ def euler_bandwidth(torch, abi):
     return res
 
 
+def token_kernels_graph(torch, abi, synth):
+    """Scheduler, re-grouping and cached Euler at the 21x30x52 and 21x45x80
+    latents ({40,20,10} at 40/30/30%), each captured as a CUDA graph of
+    back-to-back calls so the per-call figure carries no launch gaps: all 40
+    schedule calls of a loop, 20 re-groupings (score + radix select + assign),
+    100 Euler updates.  The buffers (<= 25 MB) stay in L2 across the calls."""
+    out = {}
+    stream = torch.cuda.current_stream()
+    for name in ("select_euler_32760", "select_euler_75600"):
+        spec = synth.WORKLOADS[name]
+        N, T = spec["N"], spec["T"]
+        counts = synth.group_counts(N, spec["fractions"])
+        ctx = abi.hsa_create(N=N, D=128, H=1, F=64, L=0, T=T, budgets=spec["budgets"],
+                             counts=counts)
+        vp, vc, _ = synth.velocity_pair(N, 16, spec["seed"])
+        v_prev, v_cur = torch.from_numpy(vp).cuda(), torch.from_numpy(vc).cuda()
+        g = torch.from_numpy(synth.random_split(N, counts, spec["seed"])).cuda()
+        mask = torch.zeros(N, dtype=torch.uint8, device="cuda")
+        idx = torch.zeros(N, dtype=torch.int32, device="cuda")
+        score = torch.zeros(N, dtype=torch.float32, device="cuda")
+        x, vf = (torch.randn((N, 16), device="cuda") for _ in range(2))
+        vh, vhp = v_cur.clone(), v_prev.clone()
+        gsel = g.clone()
+        calls = {
+            "schedule": (T, lambda k: abi.hsa_schedule(ctx, k % T, g, mask, idx)),
+            "regroup": (20, lambda k: abi.hsa_select_groups(ctx, v_prev, v_cur, score, gsel)),
+            "euler": (100, lambda k: abi.hsa_euler_step(ctx, x, vh, vhp, vf, mask, 0.5, 0.475)),
+        }
+        res = {}
+        for key, (n_calls, fn) in calls.items():
+            for k in range(3):
+                fn(k)
+            torch.cuda.synchronize()
+            side = torch.cuda.Stream()
+            graph = torch.cuda.CUDAGraph()
+            abi.hsa_set_stream(ctx, side)
+            try:
+                with torch.cuda.graph(graph, stream=side):
+                    for k in range(n_calls):
+                        fn(k)
+            finally:
+                abi.hsa_set_stream(ctx, None)
+            graph.replay()
+            times = []
+            for _ in range(5):
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record(stream)
+                graph.replay()
+                e1.record(stream)
+                torch.cuda.synchronize()
+                times.append(e0.elapsed_time(e1) / n_calls)
+            us = float(np.median(times)) * 1e3
+            res[key] = {"us_per_call": round(us, 2), "calls_per_graph": n_calls}
+            del graph
+        a = int(mask.sum().item())
+        eb = N * 16 * 4 * 3 + a * 16 * 4 * 3 + N
+        res["euler"]["GBps_l2_resident"] = round(eb / res["euler"]["us_per_call"] / 1e3, 1)
+        abi.hsa_sync_check(ctx)
+        ctx.close()
+        out[str(N)] = res
+    return out
+
+
 def attention_traffic():
     """DRAM bytes per launch of the attention kernel at N = |A| = 32760 from the
     committed ncu summary, or None if the kernel source changed since the capture."""
@@ -604,11 +667,14 @@ def run_ours(args, rank, world, local, pg):
     e2e_times = time_steps(loop, args.steps, torch, per_step_hook=e2e_hook)
     e2e_ms = max_over_ranks(float(np.sum(e2e_times)), pg, torch.device("cuda", local)) / args.steps
 
+    # sub-benchmarks: one GPU only (with N ranks, rank 0 alone would hold the
+    # others at teardown for minutes)
     sub = {}
-    if not args.quick and rank == 0:
+    if not args.quick and world == 1:
         sub["attention"] = attention_sweep(torch, abi, synth)
         sub["gemm"] = gemm_sweep(torch, abi)
         sub["euler"] = euler_bandwidth(torch, abi)
+        sub["token_kernels_graph"] = token_kernels_graph(torch, abi, synth)
         sub["bandwidth"] = bandwidth_sweep(torch, abi)
         sub["conditioned_layer"] = conditioned_layer(torch, abi)
         sub["presets_dit30"] = preset_sweep(torch, synth, spec, layers, loop.model._keep[0],
