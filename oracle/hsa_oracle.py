@@ -362,13 +362,18 @@ def regroup_from(T: int, budgets: Sequence[int]) -> int:
 def run_loop(weights: dict, x0: np.ndarray, g0: np.ndarray, T: int,
              budgets: Sequence[int], counts: Sequence[int], sigmas: np.ndarray,
              H: int, m: int = 0, regroup: bool = True, emulate_bf16: bool = False,
-             log: Optional[list] = None) -> np.ndarray:
+             log: Optional[list] = None, mods=None, cross=None) -> np.ndarray:
     """The HSA denoising loop over T global iterations ([TS] 2.1-2.4).
 
     Per iteration i: A_i from the schedule; embed the active latent rows; every
     layer on A_i with its own KV cache; head -> fresh velocities of A_i; cached
     Euler over all N; then (from ``regroup_from``) re-select the groups from
     the two cached velocities.  Returns x_T (float64 [N, C]).
+
+    Conditioned blocks (reading of a real video DiT, see ``layer_forward``):
+    ``mods[i][l]`` is layer l's [6, D] modulation at iteration i (it follows
+    the timestep, so it changes with i), ``cross[l]`` layer l's text
+    cross-attention; either may be None.
     """
     N, C = x0.shape
     D = weights["w_in"].shape[0]
@@ -387,7 +392,9 @@ def run_loop(weights: dict, x0: np.ndarray, g0: np.ndarray, T: int,
         idx = active_index(mask)
         h[idx] = embed(weights["w_in"], x[idx])
         for l in range(L):
-            layer_forward(weights["layers"][l], h, idx, kc[l], vc[l], H, emulate_bf16)
+            layer_forward(weights["layers"][l], h, idx, kc[l], vc[l], H, emulate_bf16,
+                          mod=None if mods is None else mods[i][l],
+                          cross=None if cross is None else cross[l])
         v_fresh = np.zeros((N, C))
         v_fresh[idx] = head(weights["w_head"], h[idx])
         x, v_hat, v_hat_prev = euler_step(x, v_hat, v_hat_prev, v_fresh, mask,

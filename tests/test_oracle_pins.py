@@ -540,3 +540,53 @@ def test_planted_mistakes_are_caught(monkeypatch):
     with pytest.raises(AssertionError):
         test_attention_textbook_loops()
     monkeypatch.setattr(O, "attention", orig_att)
+
+
+def _cond_model(seed):
+    sh = synth.ModelShape(N=24, C=16, D=8, H=2, F=16, L=2)
+    w = synth.model_weights(sh, seed)
+    w = {"w_in": w["w_in"].astype(np.float64), "w_head": w["w_head"].astype(np.float64),
+         "layers": [{k: v.astype(np.float64) for k, v in lw.items()} for lw in w["layers"]]}
+    return sh, w
+
+
+def test_conditioned_loop_neutral_is_the_plain_loop():
+    """Neutral modulation at every iteration and cross-attention whose output
+    projection is zero leave the whole loop bit for bit as the plain loop."""
+    sh, w = _cond_model(21)
+    T, budgets, counts = 8, [8, 4, 2], [8, 8, 8]
+    x0 = synth.latent(sh.N, 16, 21)
+    g0 = synth.random_split(sh.N, counts, 21)
+    sig = O.sigma_schedule(T, 1.0)
+    neutral = np.zeros((6, sh.D))
+    neutral[2] = neutral[5] = 1.0
+    mods = [[neutral] * sh.L for _ in range(T)]
+    cross = []
+    for l in range(sh.L):
+        c = synth.cross_attention_weights(sh.D, 5, 21 + l)
+        c = {k: v.astype(np.float64) for k, v in c.items()}
+        c["w_o"] = np.zeros_like(c["w_o"])
+        cross.append(c)
+    plain = O.run_loop(w, x0, g0, T, budgets, counts, sig, sh.H)
+    cond = O.run_loop(w, x0, g0, T, budgets, counts, sig, sh.H, mods=mods, cross=cross)
+    assert (plain == cond).all()
+
+
+def test_conditioned_loop_uses_each_iterations_modulation_at_that_iteration():
+    """Modulation that departs from neutral only at the last iteration leaves
+    every earlier iterate unchanged and changes the last one."""
+    sh, w = _cond_model(22)
+    T, budgets, counts = 8, [8, 4], [12, 12]
+    x0 = synth.latent(sh.N, 16, 22)
+    g0 = synth.random_split(sh.N, counts, 22)
+    sig = O.sigma_schedule(T, 1.0)
+    neutral = np.zeros((6, sh.D))
+    neutral[2] = neutral[5] = 1.0
+    mods = [[neutral] * sh.L for _ in range(T)]
+    mods[T - 1] = [synth.modulation(sh.D, 22 + l).astype(np.float64) for l in range(sh.L)]
+    la, lb = [], []
+    O.run_loop(w, x0, g0, T, budgets, counts, sig, sh.H, log=la)
+    O.run_loop(w, x0, g0, T, budgets, counts, sig, sh.H, log=lb, mods=mods)
+    for i in range(T - 1):
+        assert (la[i]["x"] == lb[i]["x"]).all()
+    assert not (la[T - 1]["x"] == lb[T - 1]["x"]).all()
