@@ -570,6 +570,38 @@ def graph_replay(torch, synth, loop, x0, g0, eager_ms):
     return out
 
 
+def conditioned_loop(torch, abi, loop, x0, g0, eager_ms):
+    """The 30-layer DiT loop with conditioned blocks: every layer modulated
+    with vectors that change each iteration, and cross-attention to 512 text
+    tokens in every layer; ms per step over the whole 40-step loop."""
+    T, L, D, n_txt = loop.T, loop.L, loop.D, 512
+    g = torch.Generator(device="cuda")
+    g.manual_seed(13)
+    rnd = lambda *sh, s=1.0: (torch.randn(sh, generator=g, device="cuda") * s)
+    mods = []
+    for i in range(T):
+        row = []
+        for l in range(L):
+            m = rnd(6, D, s=0.3)
+            m[2] += 1.0
+            m[5] += 1.0
+            row.append(m.contiguous())
+        mods.append(row)
+    xa = [abi.cross_attn(rnd(D, D, s=D ** -0.5).to(torch.bfloat16),
+                         rnd(D, D, s=D ** -0.5).to(torch.bfloat16),
+                         rnd(n_txt, D).to(torch.bfloat16), rnd(n_txt, D).to(torch.bfloat16), n_txt)
+          for _ in range(L)]
+    conds = [abi.StepCond(mods[i], xa) for i in range(T)]
+    loop.reset(x0, g0)
+    loop.step(0, True, cond=conds[0])
+    loop.reset(x0, g0)
+    ts = time_steps(loop, T, torch, per_step_hook=lambda k, i: loop.step(i, True, cond=conds[i]))
+    abi.hsa_sync_check(loop.ctx)
+    ms = float(np.mean(ts))
+    return {"n_txt": n_txt, "ms_per_step": round(ms, 3), "plain_ms_per_step": round(eager_ms, 3),
+            "overhead": round(ms / eager_ms - 1.0, 4)}
+
+
 def cpu_baseline(spec, n_rows=64, target_s=12.0):
     """The oracle on the host cores, on a bounded sample: one layer of the
     30-layer DiT for `n_rows` active rows against the full N = 32760 cache,
@@ -680,6 +712,7 @@ def run_ours(args, rank, world, local, pg):
         sub["presets_dit30"] = preset_sweep(torch, synth, spec, layers, loop.model._keep[0],
                                             loop.model._keep[1])
         sub["dit40"] = dit40_steps(torch, synth)
+        sub["conditioned_loop"] = conditioned_loop(torch, abi, loop, x0, g0, ms_step)
         sub["cuda_graph"] = graph_replay(torch, synth, loop, x0, g0, ms_step)
 
     result = None

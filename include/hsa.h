@@ -331,6 +331,29 @@ hsa_status hsa_step(hsa_ctx* ctx, const hsa_model_weights* w, const hsa_state* s
                     float sigma_i, float sigma_next, int regroup);
 
 /*
+ * Conditioning of one iteration for hsa_step_cond: per layer, the modulation
+ * vectors of this iteration (they follow the timestep, so the caller passes
+ * new ones each iteration) and the text cross-attention (fixed for the run).
+ * See hsa_layer_forward_cond for what they do; the pages give no
+ * architecture for either ([TS] 2.2 step 4 only says skipped tokens incur no
+ * cross-attention).
+ */
+typedef struct {
+  const float* const* mod;  /* host array of L device pointers, fp32 [6, D] each (a NULL
+                               entry: that layer unmodulated), or NULL for none */
+  const hsa_cross_attn* xa; /* host array of L entries, or NULL for no cross-attention */
+} hsa_cond;
+
+/*
+ * hsa_step with conditioned blocks: every layer runs hsa_layer_forward_cond
+ * with cond->mod[l] and cond->xa[l].  cond == NULL is hsa_step.  Arrays are
+ * read during the call only.  Errors as hsa_step and hsa_layer_forward_cond.
+ */
+hsa_status hsa_step_cond(hsa_ctx* ctx, const hsa_model_weights* w, const hsa_state* s,
+                         const hsa_cond* cond, int i, float sigma_i, float sigma_next,
+                         int regroup);
+
+/*
  * Group selection without any device allocation.  The paper has no
  * counterpart: this is a service for callers that cannot call cudaMalloc,
  * such as a host framework that owns all device memory through its own pool

@@ -21,7 +21,8 @@ SYMBOLS = [
     "hsa_selftest_timeout", "hsa_kernel_launches", "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
     "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_linear", "hsa_kv_scatter", "hsa_kv_scatter_packed",
     "hsa_attention", "hsa_attention_kv", "hsa_out_proj_residual", "hsa_mlp_residual",
-    "hsa_layer_forward", "hsa_layer_forward_cond", "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_step", "hsa_select_groups_static",
+    "hsa_layer_forward", "hsa_layer_forward_cond", "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_step", "hsa_step_cond",
+    "hsa_select_groups_static",
 ]
 
 STATUS = {0: "HSA_OK", 1: "HSA_ERR_INVALID_ARG", 2: "HSA_ERR_BUDGET", 3: "HSA_ERR_SHAPE",
@@ -50,6 +51,10 @@ class hsa_layer_weights(ctypes.Structure):
 class hsa_cross_attn(ctypes.Structure):
     _fields_ = [("w_q", ctypes.c_void_p), ("w_o", ctypes.c_void_p), ("k_txt", ctypes.c_void_p),
                 ("v_txt", ctypes.c_void_p), ("n_txt", ctypes.c_int)]
+
+
+class hsa_cond(ctypes.Structure):
+    _fields_ = [("mod", ctypes.POINTER(ctypes.c_void_p)), ("xa", ctypes.POINTER(hsa_cross_attn))]
 
 
 class hsa_model_weights(ctypes.Structure):
@@ -109,6 +114,8 @@ def load() -> ctypes.CDLL:
         "hsa_head": (I, [P, P, P, P, I, P]),
         "hsa_euler_step": (I, [P, P, P, P, P, P, F, F]),
         "hsa_step": (I, [P, ctypes.POINTER(hsa_model_weights), ctypes.POINTER(hsa_state), I, F, F, I]),
+        "hsa_step_cond": (I, [P, ctypes.POINTER(hsa_model_weights), ctypes.POINTER(hsa_state),
+                              ctypes.POINTER(hsa_cond), I, F, F, I]),
         "hsa_select_groups_static": (I, [P, P, I, ctypes.POINTER(I), I, P, P]),
     }
     for name, (res, args) in sig.items():
@@ -319,6 +326,30 @@ def hsa_step(ctx: Context, model: ModelBinding, i: int, sigma_i: float, sigma_ne
              regroup: bool = True) -> None:
     _check(ctx.ptr, load().hsa_step(ctx.ptr, ctypes.byref(model.weights), ctypes.byref(model.state),
                                     i, float(sigma_i), float(sigma_next), 1 if regroup else 0))
+
+
+class StepCond:
+    """The ctypes arrays of one iteration's conditioning (keeps them alive).
+
+    mods: a list of L device fp32 [6, D] tensors (None entries allowed) or
+    None; cross: a list of L hsa_cross_attn structs (see cross_attn) or None."""
+
+    def __init__(self, mods=None, cross=None):
+        self._mods = None if mods is None else (ctypes.c_void_p * max(len(mods), 1))(
+            *[None if m is None else _p(m) for m in mods])
+        self._cross = None if cross is None else (hsa_cross_attn * max(len(cross), 1))(*cross)
+        self.struct = hsa_cond(
+            ctypes.cast(self._mods, ctypes.POINTER(ctypes.c_void_p)) if mods is not None else None,
+            ctypes.cast(self._cross, ctypes.POINTER(hsa_cross_attn)) if cross is not None else None)
+        self._keep = (mods, cross)
+
+
+def hsa_step_cond(ctx: Context, model: ModelBinding, cond: Optional[StepCond], i: int,
+                  sigma_i: float, sigma_next: float, regroup: bool = True) -> None:
+    _check(ctx.ptr, load().hsa_step_cond(
+        ctx.ptr, ctypes.byref(model.weights), ctypes.byref(model.state),
+        ctypes.byref(cond.struct) if cond is not None else None, i, float(sigma_i),
+        float(sigma_next), 1 if regroup else 0))
 
 
 def hsa_select_groups_static(v_prev, v_cur, N: int, counts: Sequence[int], g, stream=None) -> None:

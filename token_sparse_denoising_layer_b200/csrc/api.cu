@@ -568,6 +568,12 @@ hsa_status hsa_euler_step(hsa_ctx* ctx, float* x, float* v_hat, float* v_hat_pre
 
 hsa_status hsa_step(hsa_ctx* ctx, const hsa_model_weights* w, const hsa_state* s, int i,
                     float sigma_i, float sigma_next, int regroup) {
+  return hsa_step_cond(ctx, w, s, nullptr, i, sigma_i, sigma_next, regroup);
+}
+
+hsa_status hsa_step_cond(hsa_ctx* ctx, const hsa_model_weights* w, const hsa_state* s,
+                         const hsa_cond* cond, int i, float sigma_i, float sigma_next,
+                         int regroup) {
   HSA_CHECK_CTX(ctx);
   if (w == nullptr || s == nullptr || (w->layers == nullptr && ctx->c.cfg.L > 0))
     return fail(ctx, HSA_ERR_INVALID_ARG, "weights and state must not be NULL");
@@ -576,9 +582,12 @@ hsa_status hsa_step(hsa_ctx* ctx, const hsa_model_weights* w, const hsa_state* s
   int n = 0;
   hsa_status st = hsa_schedule(ctx, i, s->g, s->mask, s->active_idx, nullptr, &n);
   if (st == HSA_OK) st = hsa_embed(ctx, w->w_in, s->x, s->active_idx, n, s->h);
-  for (int l = 0; st == HSA_OK && l < ctx->c.cfg.L; ++l)
-    st = hsa_layer_forward(ctx, &w->layers[l], s->h, s->active_idx, n, s->k_cache[l],
-                           s->v_cache[l]);
+  for (int l = 0; st == HSA_OK && l < ctx->c.cfg.L; ++l) {
+    const float* mod = (cond != nullptr && cond->mod != nullptr) ? cond->mod[l] : nullptr;
+    const hsa_cross_attn* xa = (cond != nullptr && cond->xa != nullptr) ? &cond->xa[l] : nullptr;
+    st = hsa_layer_forward_cond(ctx, &w->layers[l], mod, xa, s->h, s->active_idx, n,
+                                s->k_cache[l], s->v_cache[l]);
+  }
   if (st == HSA_OK) st = hsa_head(ctx, w->w_head, s->h, s->active_idx, n, s->v_fresh);
   if (st == HSA_OK)
     st = hsa_euler_step(ctx, s->x, s->v_hat, s->v_hat_prev, s->v_fresh, s->mask, sigma_i,

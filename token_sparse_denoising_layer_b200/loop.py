@@ -72,9 +72,15 @@ class HsaLoop:
     def n_active(self, i: int) -> int:
         return abi.hsa_n_active(self.ctx, i)
 
-    def step(self, i: int, regroup: bool = True) -> None:
-        abi.hsa_step(self.ctx, self.model, i, float(self.sigmas[i]), float(self.sigmas[i + 1]),
-                     regroup)
+    def step(self, i: int, regroup: bool = True, cond: "Optional[abi.StepCond]" = None) -> None:
+        """Iteration i; ``cond`` carries conditioned blocks' modulation and
+        cross-attention for this iteration (abi.StepCond), or None."""
+        if cond is None:
+            abi.hsa_step(self.ctx, self.model, i, float(self.sigmas[i]),
+                         float(self.sigmas[i + 1]), regroup)
+        else:
+            abi.hsa_step_cond(self.ctx, self.model, cond, i, float(self.sigmas[i]),
+                              float(self.sigmas[i + 1]), regroup)
 
     def run(self, regroup: bool = True, stop: Optional[int] = None):
         for i in range(self.T if stop is None else stop):
