@@ -52,7 +52,7 @@ def parse():
                          "(strong scaling)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the sub-benchmarks (profiling runs)")
-    ap.add_argument("--profile-case", choices=["attention", "gemm", "euler"], default=None,
+    ap.add_argument("--profile-case", choices=["attention", "gemm", "euler", "rows"], default=None,
                     help="run three launches of one kernel at the workload shape and exit")
     return ap.parse_args()
 
@@ -942,6 +942,37 @@ def profile_case(name):
         m = (torch.rand(N, device="cuda") < 0.6).to(torch.uint8)
         for _ in range(3):
             abi.hsa_euler_step(ctx, x, vh, vp, vf, m, 0.5, 0.45)
+    elif name == "rows":
+        # the HBM-bound row kernels, each on inputs larger than L2, two launches each:
+        # cached Euler over 4M tokens (1 GB of latent and velocities; the context's
+        # own scratch at the smallest width, D = 128, is 3.5 GB), the LN gather of
+        # all 32760 rows (D = 1536), and the KV scatter of 18900 rows into
+        # 75600 x 5120 caches
+        Ne = 4 * 1024 * 1024
+        ce = abi.hsa_create(N=Ne, D=128, H=1, F=64, L=0, T=40, budgets=[40, 20, 10],
+                            counts=[Ne - 2 * (Ne * 3 // 10), Ne * 3 // 10, Ne * 3 // 10])
+        x, vh, vp, vf = (rnd(Ne, 16) for _ in range(4))
+        m = (torch.rand(Ne, device="cuda") < 0.625).to(torch.uint8)
+        for _ in range(2):
+            abi.hsa_euler_step(ce, x, vh, vp, vf, m, 0.5, 0.45)
+        abi.hsa_sync_check(ce)
+        ce.close()
+        del x, vh, vp, vf, m
+        h = rnd(N, D)
+        u = torch.empty((N, D), dtype=torch.bfloat16, device="cuda")
+        idx = torch.arange(N, dtype=torch.int32, device="cuda")
+        for _ in range(2):
+            abi.hsa_ln_gather(ctx, h, idx, N, u)
+        del h, u, idx
+        Nk, Dk, a = 75600, 5120, 18900
+        ck = abi.hsa_create(N=Nk, D=Dk, H=40, F=64, L=1, T=1, budgets=[1], counts=[Nk])
+        kr, vr = (rnd(a, Dk).to(torch.bfloat16) for _ in range(2))
+        kc, vc = (torch.zeros((Nk, Dk), dtype=torch.bfloat16, device="cuda") for _ in range(2))
+        ik = torch.sort(torch.randperm(Nk, generator=g, device="cuda")[:a]).values.to(torch.int32)
+        for _ in range(2):
+            abi.hsa_kv_scatter(ck, kr, vr, ik, a, kc, vc)
+        abi.hsa_sync_check(ck)
+        ck.close()
     abi.hsa_sync_check(ctx)
     ctx.close()
     return 0
