@@ -279,6 +279,137 @@ __global__ void __launch_bounds__(kSelThreads) k_radix_cut(const float* __restri
   }
 }
 
+// The same cut search with a cluster of kCutCluster CTAs per cut.  CTA c
+// holds the high words of the contiguous index range [c span, (c+1) span) in
+// shared memory; each radix pass sums the CTAs' 256-bin histograms through
+// distributed shared memory, so every CTA takes the same bin; the index
+// tie-break adds the CTAs' counts of keys equal to the final high word in
+// rank order.  Every CTA runs the same cluster barriers, and a last one keeps
+// each CTA's shared memory alive while the others read it.
+constexpr int kCutCluster = 8;
+constexpr int kCutThreads = 512;
+constexpr int kCutSpanMax = 16384;  // keys per CTA: 64 KB of shared memory
+constexpr int kCutClusterMaxN = kCutCluster * kCutSpanMax;
+
+__device__ __forceinline__ uint32_t mapa_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+
+__device__ __forceinline__ int ld_cluster_s32(uint32_t caddr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(caddr) : "memory");
+  return v;
+}
+
+__global__ void __cluster_dims__(kCutCluster, 1, 1) __launch_bounds__(kCutThreads)
+    k_radix_cut_cluster(const float* __restrict__ score, int N, int span, CutParams cp,
+                        uint32_t* cuts, int* flag) {
+  extern __shared__ uint32_t skey[];  // [span]
+  __shared__ int hist[kRadixBins];    // this CTA's histogram, read by the cluster
+  __shared__ int ghist[kRadixBins];   // the cluster's
+  __shared__ int warp_sums[32];
+  __shared__ uint32_t s_sel[2];
+  __shared__ int s_cnt;  // keys of this CTA equal to the final high word, read by the cluster
+  const int j = blockIdx.x / kCutCluster;
+  const uint32_t crank = cluster_ctarank();
+  const int R = cp.rank[j];
+  if (R >= N) {  // empty tail groups (uniform over the cluster: no barrier is reached)
+    if (crank == 0 && threadIdx.x == 0) {
+      cuts[2 * j] = 0xFFFFFFFFu;
+      cuts[2 * j + 1] = 0xFFFFFFFFu;
+    }
+    return;
+  }
+  const int lo = min(N, static_cast<int>(crank) * span);
+  const int cnt = min(N, lo + span) - lo;
+  for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+    const float r = __ldg(score + lo + i);
+    if (!(r >= 0.f)) atomicOr(flag, DEV_BAD_SCORE);
+    skey[i] = key_hi(r);
+  }
+  uint32_t prefix = 0, pmask = 0;
+  int remaining = R;
+  for (int pass = 0; pass < 4; ++pass) {
+    const int shift = 24 - 8 * pass;
+    for (int b = threadIdx.x; b < kRadixBins; b += blockDim.x) hist[b] = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
+      const uint32_t h = skey[i];
+      if ((h & pmask) == prefix) atomicAdd(&hist[(h >> shift) & 0xFF], 1);
+    }
+    cluster_sync();  // every CTA's histogram is complete and visible
+    for (int b = threadIdx.x; b < kRadixBins; b += blockDim.x) {
+      const uint32_t a = smem_u32(&hist[b]);
+      int sum = 0;
+      for (int r = 0; r < kCutCluster; ++r) sum += ld_cluster_s32(mapa_rank(a, r));
+      ghist[b] = sum;
+    }
+    __syncthreads();
+    if (threadIdx.x < 32) {
+      // lane l owns bins 8l..8l+7
+      const int lane = threadIdx.x;
+      int loc[8];
+      int sl = 0;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        loc[t] = ghist[8 * lane + t];
+        sl += loc[t];
+      }
+      int incl = sl;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        int y = __shfl_up_sync(0xffffffffu, incl, o);
+        if (lane >= o) incl += y;
+      }
+      int cum = incl - sl;
+#pragma unroll
+      for (int t = 0; t < 8; ++t) {
+        if (cum <= remaining && remaining < cum + loc[t]) {
+          s_sel[0] = static_cast<uint32_t>(8 * lane + t);
+          s_sel[1] = static_cast<uint32_t>(cum);
+        }
+        cum += loc[t];
+      }
+    }
+    __syncthreads();
+    const uint32_t bin = s_sel[0];
+    remaining -= static_cast<int>(s_sel[1]);
+    prefix |= bin << shift;
+    pmask |= 0xFFu << shift;
+    cluster_sync();  // no CTA clears its histogram while another still reads it
+  }
+  // tie-break by index: the remaining-th key (0-based) whose high word is prefix
+  int eq_local = 0;
+  for (int i = threadIdx.x; i < cnt; i += blockDim.x) eq_local += (skey[i] == prefix) ? 1 : 0;
+  const int eq_cta = block_sum(eq_local, warp_sums);
+  if (threadIdx.x == 0) s_cnt = eq_cta;
+  cluster_sync();
+  int before = 0;
+  {
+    const uint32_t a = smem_u32(&s_cnt);
+    for (uint32_t r = 0; r < crank; ++r) before += ld_cluster_s32(mapa_rank(a, r));
+  }
+  cluster_sync();  // all counts have been read: CTAs may now leave
+  if (remaining >= before && remaining < before + eq_cta) {
+    const int want = remaining - before;
+    int running = 0;
+    for (int base = 0; base < cnt; base += blockDim.x) {
+      const int i = base + threadIdx.x;
+      const int eq = (i < cnt && skey[i] == prefix) ? 1 : 0;
+      int total;
+      const int pos = running + block_exclusive_scan(eq, warp_sums, &total);
+      if (eq && pos == want) {
+        cuts[2 * j] = prefix;
+        cuts[2 * j + 1] = static_cast<uint32_t>(lo + i);
+      }
+      running += total;
+      if (running > want) break;  // uniform across the block
+    }
+  }
+}
+
 __global__ void __launch_bounds__(256) k_assign(const float* __restrict__ score,
                                                 const uint32_t* __restrict__ cuts, int ncut,
                                                 uint8_t* __restrict__ g, int N) {
@@ -309,9 +440,19 @@ cudaError_t launch_select(const Ctx& c, const float* score, uint8_t* g) {
     acc += c.counts[j];
     cp.rank[j] = acc;
   }
-  k_radix_cut<<<ncut, kSelThreads, 0, c.stream>>>(score, N, cp, c.cuts, c.flag);
+  cudaError_t e;
+  if (N <= kCutClusterMaxN) {
+    static std::atomic<uint64_t> smem_set{0};  // per device
+    e = ensure_smem_limit(k_radix_cut_cluster, kCutSpanMax * 4, c.device, smem_set);
+    if (e != cudaSuccess) return e;
+    const int span = (N + kCutCluster - 1) / kCutCluster;
+    k_radix_cut_cluster<<<ncut * kCutCluster, kCutThreads, span * 4, c.stream>>>(
+        score, N, span, cp, c.cuts, c.flag);
+  } else {
+    k_radix_cut<<<ncut, kSelThreads, 0, c.stream>>>(score, N, cp, c.cuts, c.flag);
+  }
   c.launches += 2;  // with k_assign below
-  cudaError_t e = cudaGetLastError();
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   k_assign<<<(N + 255) / 256, 256, 0, c.stream>>>(score, c.cuts, ncut, g, N);
   return cudaGetLastError();
