@@ -232,7 +232,7 @@ def euler_bandwidth(torch, abi):
     """Cached-Euler kernel GB/s at the 21x30x52 and 21x45x80 latents (L2 flushed
     between samples) and at a 256M-float size (asymptotic)."""
     res = {}
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush = _l2_flush(torch)
     stream = torch.cuda.current_stream()
     for N in (32760, 75600, 16 * 1024 * 1024):
         ctx = abi.hsa_create(N=N, D=128, H=1, F=64, L=0, T=40, budgets=[40, 20, 10],
@@ -242,7 +242,7 @@ def euler_bandwidth(torch, abi):
         a = int(mask.sum().item())
         times = []
         for r in range(13):
-            flush.fill_(float(r))
+            _do_flush(flush, r)
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             abi.hsa_euler_step(ctx, x, vh, vp, vf, mask, 0.5, 0.475)
@@ -340,16 +340,32 @@ def attention_traffic():
         return None
 
 
+def _l2_flush(torch):
+    """Two 256 MB buffers: one written between samples (evicts every line), then
+    one read, so the written lines are back in HBM before the sample starts and
+    the timed kernel pays for no one else's write-back."""
+    n = 256 * 1024 * 1024 // 4
+    return (torch.empty(n, dtype=torch.float32, device="cuda"),
+            torch.ones(n, dtype=torch.float32, device="cuda"))
+
+
+def _do_flush(flush, r):
+    wbuf, rbuf = flush
+    wbuf.fill_(float(r))
+    rbuf.sum()
+
+
 def _time(fn, torch, reps=10, flush=None):
     """Median CUDA-event time (ms) of fn() on the current stream, after warm-up;
-    with `flush`, a 256 MB buffer is written between samples (cold L2)."""
+    with `flush` (see _l2_flush), L2 holds neither useful nor dirty lines when
+    each sample starts."""
     stream = torch.cuda.current_stream()
     for _ in range(3):
         fn()
     times = []
     for r in range(reps):
         if flush is not None:
-            flush.fill_(float(r))
+            _do_flush(flush, r)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         fn()
@@ -384,7 +400,7 @@ def gemm_sweep(torch, abi):
 def bandwidth_sweep(torch, abi):
     """HBM-bound row kernels at the workloads' sizes, L2 flushed between samples:
     the standalone KV-cache scatter (dit30 and dit40 shapes) and the LN gather."""
-    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device="cuda")
+    flush = _l2_flush(torch)
     res = {}
     for name, N, D, a in (("kv_scatter_dit30_f1", 32760, 1536, 32760),
                           ("kv_scatter_dit40_f0.25", 75600, 5120, 18900)):
