@@ -161,6 +161,13 @@ def test_cond_argument_errors():
     with pytest.raises(abi.HsaError) as e:
         abi.hsa_layer_forward_cond(ctx, lw, mod[1:], None, x, idx, 4, kc, kc.clone())
     assert e.value.status == 1
+    # a misaligned text-key pointer is refused on the host, before any launch
+    k_txt = bf(cross["k_txt"])
+    xa2 = _device_cross(cross)
+    xa2.k_txt = k_txt.data_ptr() + 2
+    with pytest.raises(abi.HsaError) as e:
+        abi.hsa_layer_forward_cond(ctx, lw, None, xa2, x, idx, 4, kc, kc.clone())
+    assert e.value.status == 1
     ctx.close()
 
 

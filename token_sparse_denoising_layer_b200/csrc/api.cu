@@ -494,8 +494,10 @@ hsa_status hsa_layer_forward_cond(hsa_ctx* ctx, const hsa_layer_weights* w, cons
     return fail(ctx, HSA_ERR_INVALID_ARG, "mod must be 16-byte aligned");
   if (xa != nullptr) {
     if (xa->n_txt <= 0) return fail(ctx, HSA_ERR_SHAPE, "cross-attention needs n_txt >= 1");
-    if (!xa->w_q || !xa->w_o || !xa->k_txt || !xa->v_txt)
-      return fail(ctx, HSA_ERR_INVALID_ARG, "cross-attention pointer is NULL");
+    HSA_CHECK_PTR(ctx, xa->w_q);
+    HSA_CHECK_PTR(ctx, xa->w_o);
+    HSA_CHECK_PTR(ctx, xa->k_txt);
+    HSA_CHECK_PTR(ctx, xa->v_txt);
   }
   if (n == 0) return HSA_OK;
   Ctx& c = ctx->c;
