@@ -618,6 +618,51 @@ def conditioned_loop(torch, abi, loop, x0, g0, eager_ms):
             "overhead": round(ms / eager_ms - 1.0, 4)}
 
 
+def oracle_beside(reps=3):
+    """The oracle on the host cores for the smaller workloads, timed in the same
+    run as the GPU figures for the same work: the whole tiny-DiT loop (ms per
+    step), and one re-grouping (score + ranking) and one cached-Euler update at
+    N = 32760 (ms per call).  Median of `reps`."""
+    from oracle import hsa_oracle as O
+    from token_sparse_denoising_layer_b200 import synth
+
+    def med(fn):
+        ts = []
+        for _ in range(reps):
+            t0 = time.perf_counter()
+            fn()
+            ts.append(time.perf_counter() - t0)
+        return float(np.median(ts)) * 1e3
+
+    spec = synth.WORKLOADS["tiny_dit"]
+    sh = spec["shape"]
+    counts = synth.group_counts(sh.N, spec["fractions"])
+    w = synth.model_weights(sh, 0)
+    x0 = synth.latent(sh.N, 16, 0)
+    g0 = synth.random_split(sh.N, counts, 0)
+    sig = O.sigma_schedule(spec["T"], spec["shift"])
+    tiny = med(lambda: O.run_loop(w, x0, g0, spec["T"], list(spec["budgets"]), counts, sig,
+                                  sh.H)) / spec["T"]
+    s2 = synth.WORKLOADS["select_euler_32760"]
+    N = s2["N"]
+    vp, vc, _ = synth.velocity_pair(N, 16, s2["seed"])
+    c2 = synth.group_counts(N, s2["fractions"])
+    regroup = med(lambda: O.assign_groups(O.l1_relative_change(vp, vc), c2))
+    r = synth.rng(3)
+    x, vf = (r.standard_normal((N, 16)) for _ in range(2))
+    mask = r.random(N) < 0.625
+    euler = med(lambda: O.euler_step(x, vc, vp, vf, mask, 0.5, 0.475))
+    try:
+        import torch
+        cores = torch.get_num_threads()
+    except Exception:
+        cores = os.cpu_count()
+    return {"cores": cores, "kind": "oracle",
+            "tiny_dit_loop_ms_per_step": round(tiny, 3),
+            "regroup_32760_ms": round(regroup, 3),
+            "euler_32760_ms": round(euler, 3)}
+
+
 def cpu_baseline(spec, n_rows=64, target_s=12.0):
     """The oracle on the host cores, on a bounded sample: one layer of the
     30-layer DiT for `n_rows` active rows against the full N = 32760 cache,
@@ -783,6 +828,11 @@ def run_ours(args, rank, world, local, pg):
         }
         if not args.no_cpu_baseline and world == 1:
             result["cpu_baseline"] = cpu_baseline(spec)
+            if sub:
+                # the oracle beside the GPU on the smaller workloads; the GPU
+                # figures for the same work are sub.cuda_graph.tiny_dit and
+                # sub.token_kernels_graph["32760"]
+                sub["oracle_beside"] = oracle_beside()
     loop.close()
     return result
 

@@ -51,3 +51,13 @@ def test_help_lists_the_contract_flags():
     assert r.returncode == 0
     for flag in ("--gpus", "--steps", "--warmup", "--impl", "--mode"):
         assert flag in r.stdout
+
+
+def test_oracle_beside_times_the_small_workloads():
+    sys.path.insert(0, ROOT)
+    import bench
+
+    d = bench.oracle_beside(reps=1)
+    assert d["kind"] == "oracle" and d["cores"] >= 1
+    for k in ("tiny_dit_loop_ms_per_step", "regroup_32760_ms", "euler_32760_ms"):
+        assert d[k] > 0
