@@ -409,6 +409,53 @@ def test_cross_attention_textbook_and_closed_form():
     assert np.allclose(tr2["oc"], np.tile(c["v_txt"].mean(axis=0), (len(idx), 1)), atol=1e-12)
 
 
+# ---------------------------------------------------------------- embed and velocity head
+
+def _lin_loops(W, v):
+    return [math.fsum(W[o][t] * v[t] for t in range(len(v))) for o in range(len(W))]
+
+
+def test_embed_textbook_loops_and_one_hot_rows():
+    """Patch embed, latent rows [a, C] -> hidden rows [a, D] with w_in [D, C]:
+    hidden value o of a row is the dot product of the row with w_in's row o.
+    Checked with loops, once with D = C = 16 (where a transposed w_in keeps the
+    right shape), and on one-hot latent rows, which pick out one column of w_in."""
+    r = np.random.default_rng(30)
+    for D in (16, 8):
+        w_in = r.standard_normal((D, 16))
+        xl = r.standard_normal((5, 16)) * 2.0
+        got = O.embed(w_in, xl)
+        want = np.array([_lin_loops(w_in.tolist(), row) for row in xl.tolist()])
+        assert got.shape == (5, D)
+        assert np.allclose(got, want, atol=1e-12)
+    w_in = r.standard_normal((16, 16))
+    onehot = np.eye(16)[[0, 5, 15]]
+    assert np.array_equal(O.embed(w_in, onehot), w_in[:, [0, 5, 15]].T)
+
+
+def test_head_textbook_loops_and_closed_forms():
+    """Velocity head, hidden rows [a, D] -> velocities [a, C] with w_head [C, D]:
+    the final LayerNorm of the row (no affine, eps 1e-5), then the linear map.
+    Checked with loops (D = C = 16, so a transposed w_head keeps the shape); a
+    constant row normalises to zero and so predicts zero velocity; a positive
+    affine change of a row leaves the prediction as it was; a row that already
+    has zero mean and unit variance is only divided by sqrt(1 + eps)."""
+    r = np.random.default_rng(31)
+    for D in (16, 24):
+        w_head = r.standard_normal((16, D))
+        h = r.standard_normal((5, D)) * 3.0 + 1.5
+        got = O.head(w_head, h)
+        want = np.array([_lin_loops(w_head.tolist(), _ln_loops(row)) for row in h.tolist()])
+        assert got.shape == (5, 16)
+        assert np.allclose(got, want, atol=1e-11)
+    w_head = r.standard_normal((16, 24))
+    assert np.allclose(O.head(w_head, np.full((3, 24), 4.25)), 0.0, atol=1e-12)
+    h = r.standard_normal((4, 24))
+    assert np.allclose(O.head(w_head, 5.0 * h - 2.0), O.head(w_head, h), atol=1e-5)
+    z = np.array([[1.0, -1.0] * 12])                    # mean 0, variance 1
+    assert np.allclose(O.head(w_head, z), (z @ w_head.T) / math.sqrt(1.0 + 1e-5), atol=1e-13)
+
+
 # ---------------------------------------------------------------- cached Euler (2.3)
 
 def test_euler_telescoping_closed_form():
@@ -512,8 +559,10 @@ def test_loop_regroup_keeps_counts():
 # ---------------------------------------------------------------- planted mistakes
 
 def test_planted_mistakes_are_caught(monkeypatch):
-    """A wrong sign in the Euler step, a transposed key operand and a dropped
-    eps each break one of the pins above."""
+    """A wrong sign in the Euler step, values paired with the wrong keys, a
+    dropped LN eps, a head without its final LayerNorm or with w_head transposed,
+    and an embed with w_in transposed or its output scaled each break one of the
+    pins above."""
     orig_euler = O.euler_step
 
     def bad_euler(x, vh, vp, vf, mask, si, sn):
@@ -540,6 +589,28 @@ def test_planted_mistakes_are_caught(monkeypatch):
     with pytest.raises(AssertionError):
         test_attention_textbook_loops()
     monkeypatch.setattr(O, "attention", orig_att)
+
+    orig_head = O.head
+    monkeypatch.setattr(O, "head", lambda w_head, h: np.asarray(h) @ np.asarray(w_head).T)
+    with pytest.raises(AssertionError):                  # final LayerNorm dropped
+        test_head_textbook_loops_and_closed_forms()
+    monkeypatch.setattr(O, "head", lambda w_head, h: orig_head(np.asarray(w_head).T, h)
+                        if np.asarray(w_head).shape[0] == np.asarray(w_head).shape[1]
+                        else orig_head(w_head, h))
+    with pytest.raises(AssertionError):                  # w_head transposed
+        test_head_textbook_loops_and_closed_forms()
+    monkeypatch.setattr(O, "head", orig_head)
+
+    orig_embed = O.embed
+    monkeypatch.setattr(O, "embed", lambda w_in, xl: orig_embed(np.asarray(w_in).T, xl)
+                        if np.asarray(w_in).shape[0] == np.asarray(w_in).shape[1]
+                        else orig_embed(w_in, xl))
+    with pytest.raises(AssertionError):                  # w_in transposed
+        test_embed_textbook_loops_and_one_hot_rows()
+    monkeypatch.setattr(O, "embed", lambda w_in, xl: 2.0 * orig_embed(w_in, xl))
+    with pytest.raises(AssertionError):                  # output scaled
+        test_embed_textbook_loops_and_one_hot_rows()
+    monkeypatch.setattr(O, "embed", orig_embed)
 
 
 def _cond_model(seed):
