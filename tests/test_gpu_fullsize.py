@@ -1,17 +1,21 @@
 """Parity at the workloads' full sizes, in the launch configuration bench.py
 times (hsa_layer_forward / hsa_step), checked on sampled outputs the oracle
-computes one by one.
+computes one by one (tests/sampled_block.py, itself checked against the
+oracle's whole block on small cases).
 
-The oracle builds the exact KV cache the sampled queries see: every active
-row's fresh K and V (float64), stale rows elsewhere.  Then, for sampled active
-rows, it runs attention against that cache and the rest of the block.
-Skipped rows of x and of the caches must be untouched, bit for bit.
+Where the oracle can afford it, it builds the exact KV cache the sampled
+queries see: every active row's fresh K and V (float64), stale rows elsewhere.
+For the 40-layer DiT's layer at 25% and 100% active (18900 and 75600 of 75600
+rows at D = 5120) it checks the GPU's fresh K/V rows on a sample first, then
+attends against the cache as the GPU wrote it.  Skipped rows of x and of the
+caches must be untouched, bit for bit.
 """
 
 import numpy as np
 import pytest
 
 from gpu_util import BF16_TOL, bf, dev, host, need_gpu, normwise, torch
+import sampled_block as SB
 from oracle import hsa_oracle as O
 from token_sparse_denoising_layer_b200 import abi, synth
 
@@ -23,29 +27,17 @@ def _device_weights(D, F, seed):
     return w, abi.layer_weights(*(bf(w[k]) for k in ("w_qkv", "w_o", "w_1", "w_2")))
 
 
-def _sampled_block_reference(w, x, idx, ks, vs, H, rows):
-    """Oracle block outputs for the active rows idx[rows], given the full cache update."""
-    D = x.shape[1]
-    u = O.layer_norm(x[idx])                               # all active rows: K, V into the cache
-    kv = O.linear(u, w["w_qkv"][D:])
-    kc = ks.astype(np.float64)
-    vc = vs.astype(np.float64)
-    kc[idx] = kv[:, :D]
-    vc[idx] = kv[:, D:]
-    q = O.linear(u[rows], w["w_qkv"][:D])
-    o = O.attention(q, kc, vc, H)
-    x1 = x[idx[rows]].astype(np.float64) + O.linear(o, w["w_o"])
-    x2 = x1 + O.linear(O.gelu(O.linear(O.layer_norm(x1), w["w_1"])), w["w_2"])
-    return x2, kc[idx[rows]], vc[idx[rows]]
-
-
-@pytest.mark.parametrize("name,N,D,H,F,a,n_sample", [
-    ("layer_1536 f=1", 32760, 1536, 12, 6144, 32760, 192),
-    ("layer_1536 f=0.1", 32760, 1536, 12, 6144, 3276, 192),
-    ("dit30 layer, 40% active", 32760, 1536, 12, 8960, 13104, 128),
-    ("dit40 layer, 2048 active", 75600, 5120, 40, 13824, 2048, 48),
+@pytest.mark.parametrize("name,N,D,H,F,a,n_sample,via_gpu_cache", [
+    ("layer_1536 f=1", 32760, 1536, 12, 6144, 32760, 192, False),
+    ("layer_1536 f=0.5", 32760, 1536, 12, 6144, 16380, 128, False),
+    ("layer_1536 f=0.25", 32760, 1536, 12, 6144, 8190, 128, False),
+    ("layer_1536 f=0.1", 32760, 1536, 12, 6144, 3276, 192, False),
+    ("dit30 layer, 40% active", 32760, 1536, 12, 8960, 13104, 128, False),
+    ("dit40 layer, 2048 active", 75600, 5120, 40, 13824, 2048, 48, False),
+    ("dit40 layer, 25% active", 75600, 5120, 40, 13824, 18900, 64, True),
+    ("dit40 layer, 100% active", 75600, 5120, 40, 13824, 75600, 64, True),
 ])
-def test_layer_full_size_sampled(name, N, D, H, F, a, n_sample):
+def test_layer_full_size_sampled(name, N, D, H, F, a, n_sample, via_gpu_cache):
     need_gpu()
     ctx = abi.hsa_create(N=N, D=D, H=H, F=F, L=1, T=1, budgets=[1], counts=[N])
     w, lw = _device_weights(D, F, 21)
@@ -62,12 +54,25 @@ def test_layer_full_size_sampled(name, N, D, H, F, a, n_sample):
     if a - 1 not in rows:
         rows[-1] = a - 1
     rows = np.unique(rows)
-    x_ref, k_ref, v_ref = _sampled_block_reference(w, x, idx, ks, vs, H, rows)
     xg = host(xd)
     n_rows = idx[rows]
-    assert normwise(xg[n_rows] - x[n_rows], x_ref - x[n_rows]) <= BF16_TOL, name
-    assert normwise(host(kc)[n_rows], k_ref) <= BF16_TOL
-    assert normwise(host(vc)[n_rows], v_ref) <= BF16_TOL
+    if via_gpu_cache:
+        # the fresh K/V rows on a wider sample first, then attention against
+        # the cache the GPU wrote (the sampled rows of which are now checked)
+        kv_rows = np.unique(np.r_[rows, np.sort(r.choice(a, size=min(512, a), replace=False))])
+        k_ref, v_ref = SB.kv_rows(w, x, idx, kv_rows)
+        kg, vg = host(kc), host(vc)
+        assert normwise(kg[idx[kv_rows]], k_ref) <= BF16_TOL, name
+        assert normwise(vg[idx[kv_rows]], v_ref) <= BF16_TOL, name
+        x_ref = SB.block_rows_given_cache(w, x, idx, kg, vg, H, rows)
+        del kg, vg
+    else:
+        x_ref, k_ref, v_ref = SB.block_rows(w, x, idx, ks, vs, H, rows)
+        assert normwise(host(kc)[n_rows], k_ref) <= BF16_TOL
+        assert normwise(host(vc)[n_rows], v_ref) <= BF16_TOL
+    err = normwise(xg[n_rows] - x[n_rows], x_ref - x[n_rows])
+    print(f"{name}: block output error {err:.2e} on {len(rows)} sampled rows")
+    assert err <= BF16_TOL, name
     skipped = np.setdiff1d(np.arange(N), idx)
     if len(skipped):
         s = r.choice(skipped, size=min(512, len(skipped)), replace=False)
@@ -76,53 +81,39 @@ def test_layer_full_size_sampled(name, N, D, H, F, a, n_sample):
     ctx.close()
 
 
-def test_dit30_shapes_loop_drift():
-    """The whole loop at the 30-layer DiT's D, H, F, T, shift and budgets, with
-    one layer and a 21x5x8 latent (N = 840), against the float64 oracle."""
+@pytest.mark.parametrize("workload,seed,regroup", [
+    ("dit30_1536", 3, False), ("dit30_1536", 3, True), ("dit40_5120", 4, True)])
+def test_reduced_shape_loop(workload, seed, regroup):
+    """The whole loop at a large workload's D, H, F, T, shift and budgets (the
+    30-layer DiT: 1536 wide, {40, 20, 10} at 40/30/30; the 40-layer DiT: 5120
+    wide, {40, 10} at 25/75), with L = 2 layers and a 21x8x10 latent
+    (N = 1680).  Every iteration is checked
+    (loop_check.run_checked: schedule of the GPU's groups; bit-exact scores
+    and assignment at every re-grouping); x_T is compared with the float64 oracle's loop."""
     need_gpu()
-    spec = synth.WORKLOADS["dit30_1536"]
-    sh = synth.ModelShape(N=840, C=16, D=1536, H=12, F=8960, L=1)
+    from loop_check import run_checked
+    from token_sparse_denoising_layer_b200.loop import HsaLoop
+
+    spec = synth.WORKLOADS[workload]
+    big = spec["shape"]
+    sh = synth.ModelShape(N=1680, C=16, D=big.D, H=big.H, F=big.F, L=2)
     T, budgets = spec["T"], list(spec["budgets"])
     counts = synth.group_counts(sh.N, spec["fractions"])
-    w = synth.model_weights(sh, 3)
+    w = synth.model_weights(sh, seed)
     layers = [tuple(bf(lw[k]) for k in ("w_qkv", "w_o", "w_1", "w_2")) for lw in w["layers"]]
-    from token_sparse_denoising_layer_b200.loop import HsaLoop
     loop = HsaLoop(sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]), T, budgets,
                    counts, shift=spec["shift"])
-    x0 = synth.latent(sh.N, 16, 3)
-    g0 = synth.random_split(sh.N, counts, 3)
+    x0 = synth.latent(sh.N, 16, seed)
+    g0 = synth.random_split(sh.N, counts, seed)
     loop.reset(x0, g0)
-    loop.run(regroup=False)
-    abi.hsa_sync_check(loop.ctx)
+    n_regroup, moved = run_checked(loop, T, budgets, counts, g0, regroup=regroup)
+    log = []
     xr = O.run_loop(w, x0, g0, T, budgets, counts, O.sigma_schedule(T, spec["shift"]), sh.H,
-                    regroup=False)
+                    regroup=regroup, log=log)
     drift = float(np.linalg.norm(host(loop.x) - xr) / np.linalg.norm(xr))
-    print(f"dit30-shape loop (L=1, N=840, T=40) x_T drift vs float64 oracle: {drift:.3e}")
-    assert drift <= 2e-2
-    loop.close()
-
-
-def test_dit40_shapes_loop_drift():
-    """The whole loop at the 40-layer DiT's D, H, F, T, shift and budgets ({40, 10}
-    at 25/75%), with one layer and N = 210 tokens, against the float64 oracle."""
-    need_gpu()
-    spec = synth.WORKLOADS["dit40_5120"]
-    sh = synth.ModelShape(N=210, C=16, D=5120, H=40, F=13824, L=1)
-    T, budgets = spec["T"], list(spec["budgets"])
-    counts = synth.group_counts(sh.N, spec["fractions"])
-    w = synth.model_weights(sh, 4)
-    layers = [tuple(bf(lw[k]) for k in ("w_qkv", "w_o", "w_1", "w_2")) for lw in w["layers"]]
-    from token_sparse_denoising_layer_b200.loop import HsaLoop
-    loop = HsaLoop(sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]), T, budgets,
-                   counts, shift=spec["shift"])
-    x0 = synth.latent(sh.N, 16, 4)
-    g0 = synth.random_split(sh.N, counts, 4)
-    loop.reset(x0, g0)
-    loop.run(regroup=False)
-    abi.hsa_sync_check(loop.ctx)
-    xr = O.run_loop(w, x0, g0, T, budgets, counts, O.sigma_schedule(T, spec["shift"]), sh.H,
-                    regroup=False)
-    drift = float(np.linalg.norm(host(loop.x) - xr) / np.linalg.norm(xr))
-    print(f"dit40-shape loop (L=1, N=210, T=40) x_T drift vs float64 oracle: {drift:.3e}")
+    parted = int((host(loop.g) != log[-1]["g"]).sum())
+    print(f"{workload} shapes (L=2, N=1680, T={T}, regroup={regroup}): x_T drift vs float64 "
+          f"oracle {drift:.3e}; {n_regroup} re-groupings moved {moved} group ids; final "
+          f"groups differ from the oracle's on {parted} of {sh.N} tokens")
     assert drift <= 2e-2
     loop.close()

@@ -4,7 +4,12 @@ tiny DiT workload (4x8x8 latent, N=256, 2 layers, T=8, budgets {8, 4}).
 The GPU runs the layers in bf16 and the oracle in float64, so the latents
 drift apart by rounding; the drift after T steps is stated and bounded here.
 With re-grouping on, a rounding difference can move a token whose score sits
-on a group boundary, so that run is checked for valid groups and a looser drift.
+on a group boundary, so the two runs' groups may part; what is unique is
+checked step by step instead: at every iteration the GPU's active list is the
+oracle's schedule of the GPU's groups, and after every re-grouping the GPU's
+score buffer is the oracle's float32 L1 relative change of the GPU's own two
+cached velocities, bit for bit, and the GPU's groups are the oracle's
+assignment of that buffer.
 """
 
 import numpy as np
@@ -14,6 +19,7 @@ from gpu_util import bf, dev, host, need_gpu, torch
 from oracle import hsa_oracle as O
 from token_sparse_denoising_layer_b200 import abi, synth
 from token_sparse_denoising_layer_b200.loop import HsaLoop, sigma_schedule
+from loop_check import run_checked
 
 pytestmark = pytest.mark.gpu
 
@@ -36,6 +42,7 @@ def _drift(a, b):
     return float(np.linalg.norm(a - b) / np.linalg.norm(b))
 
 
+
 def test_sigma_tables_agree():
     for T, s in ((8, 1.0), (40, 5.0)):
         assert (sigma_schedule(T, s) == O.sigma_schedule(T, s)).all()
@@ -55,6 +62,22 @@ def test_tiny_dit_loop_drift(regroup):
     d = _drift(xg, xr)
     print(f"tiny DiT x_T drift vs float64 oracle (regroup={regroup}): {d:.3e}")
     assert d <= (2e-2 if not regroup else 5e-2)
+
+
+def test_tiny_dit_regrouping_exact_at_every_step():
+    """Re-grouping on, the tiny DiT loop checked iteration by iteration (see
+    ``run_checked``), then its x_T against the oracle's loop."""
+    need_gpu()
+    sh, T, counts, w, loop, x0, g0 = _setup()
+    loop.reset(x0, g0)
+    n_regroup, moved = run_checked(loop, T, [8, 4], counts, g0)
+    assert n_regroup == T - 1 - O.regroup_from(T, [8, 4])
+    assert moved > 0                      # the groups really do change
+    xr = O.run_loop(w, x0, g0, T, [8, 4], counts, O.sigma_schedule(T, 1.0), sh.H)
+    d = _drift(host(loop.x), xr)
+    print(f"tiny DiT, re-grouping checked per step: {n_regroup} re-groupings moved "
+          f"{moved} group ids; x_T drift {d:.3e}")
+    assert d <= 2e-2
 
 
 def test_all_active_loop_matches_dense_oracle():
