@@ -130,6 +130,29 @@ hsa_status hsa_selftest_timeout(hsa_ctx* ctx, int timeout_us);
 uint64_t hsa_kernel_launches(const hsa_ctx* ctx);
 
 /*
+ * Per-launch timing of the calls above, for measuring the kernels inside a
+ * running step (no counterpart on the pages: instrumentation).  While on, every
+ * kernel launch of the context is bracketed by two CUDA events on its stream
+ * and its algorithmic work is added up per class:
+ *   0 attention   (hsa_attention, hsa_attention_kv; work = 4 n n_kv D FLOP)
+ *   1 GEMM        (QKV, out-projection, MLP, linear; work = 2 M Ncols K FLOP)
+ *   2 row kernels (LN gather, KV scatter, embed, head; work = bytes moved)
+ *   3 per-token   (schedule, score, selection, Euler; work = 0)
+ * hsa_kernel_times synchronises the stream, writes the first n_classes
+ * classes' totals (launch calls, summed event milliseconds, work) to out, and
+ * clears them.  Events are taken from a pool the context owns.  Off by
+ * default; not meant for use under stream capture.
+ */
+typedef struct {
+  uint64_t calls;
+  double ms;
+  double work;
+} hsa_kernel_class_time;
+
+hsa_status hsa_time_kernels(hsa_ctx* ctx, int on);
+hsa_status hsa_kernel_times(hsa_ctx* ctx, hsa_kernel_class_time* out, int n_classes);
+
+/*
  * |A_i| computed on the host from the group counts ([TS] 2.1): the sum of n_k
  * over the groups active at iteration i.  Valid when g holds exactly counts[k]
  * tokens of group k, which the initial split and hsa_select_groups guarantee.
@@ -320,10 +343,27 @@ hsa_status hsa_euler_step(hsa_ctx* ctx, float* x, float* v_hat, float* v_hat_pre
                           float sigma_next);
 
 /*
+ * The same cached Euler update, and in the same pass the score of the
+ * re-grouping that follows it ([TS] 2.1, Dynamic Selection; [TS] 2.3): after
+ * the update above,
+ *   score[n] = sum_c |v_hat[n,c] - v_hat_prev[n,c]| / (sum_c |v_hat_prev[n,c]| + 1e-6)
+ * in float32, sums in channel order, bit for bit what hsa_score writes for
+ * (v_hat_prev, v_hat).  A re-grouping step thus reads the velocity caches
+ * once; hsa_select_from_score then assigns the groups.
+ *   score (device) fp32 [N] out; the other arguments as hsa_euler_step.
+ *   A NaN, negative or infinite score is reported by hsa_sync_check
+ *   (HSA_ERR_DEVICE_CHECK).
+ */
+hsa_status hsa_euler_step_score(hsa_ctx* ctx, float* x, float* v_hat, float* v_hat_prev,
+                                const float* v_fresh, const uint8_t* mask, float sigma_i,
+                                float sigma_next, float* score);
+
+/*
  * One global iteration i of the HSA loop ([TS] 2.1-2.3): schedule -> embed
  * the active latent rows -> every layer on A_i -> head -> cached Euler over
  * all N -> (when ``regroup`` is non-zero and T/s_K <= i < T-1) re-select the
- * groups from v_hat_prev and v_hat.  No host synchronisation.
+ * groups from v_hat_prev and v_hat (the Euler pass writes the scores, as
+ * hsa_euler_step_score).  No host synchronisation.
  *   w (host) model weights;  s (host) state;  sigma_i, sigma_next the noise
  *   levels of iterations i and i+1.
  */
@@ -363,15 +403,19 @@ hsa_status hsa_step_cond(hsa_ctx* ctx, const hsa_model_weights* w, const hsa_sta
  * Same result as hsa_select_groups (scores, then exact group assignment with
  * ties broken by token index), but it needs no context: the scores and cut
  * keys live in one static device array of the library, sized for at most
- * HSA_SELECT_STATIC_MAX_N tokens (512 KiB + 256 B), which every GPU that
- * loads the library holds until the process exits.
+ * HSA_SELECT_STATIC_MAX_N tokens (512 KiB of scores + 64 B of cut keys +
+ * 256 B for the error flag), which every GPU that loads the library holds
+ * until the process exits.
  *   v_prev, v_cur (device) fp32 [N, 16];  counts (host) n_1..n_K, sum == N;
  *   g (device) uint8 [N] out;  stream cudaStream_t (NULL = legacy default).
  * Returns HSA_ERR_SCRATCH_LIMIT when N > HSA_SELECT_STATIC_MAX_N, and the
  * other argument errors of hsa_create / hsa_select_groups; there is no
  * message string.  Calls no cudaMalloc or cudaFree.  The first call on a
  * device looks up the array's device address (cudaGetSymbolAddress) with
- * that device current; make that first call before any stream capture.
+ * that device current; make that first call before any stream capture.  The
+ * address belongs to the device's primary context: after cudaDeviceReset the
+ * next call finds a new context and looks the address up again (make that
+ * call, too, outside stream capture).
  * All calls share the array and it keeps the last call's contents; calls
  * that overlap on the GPU race on it.  Device-side checks (a NaN score) are
  * not reported by this call.

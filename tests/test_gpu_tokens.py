@@ -161,6 +161,36 @@ def test_euler_bit_exact(N):
     assert np.abs(host(xd) - fx).max() / np.abs(fx).max() <= EULER_TOL
 
 
+@pytest.mark.parametrize("N", [1, 3, 255, 4097, 32760, 75600])
+def test_euler_with_score_bit_exact(N):
+    """The Euler pass that also scores the re-grouping: x and both caches as
+    hsa_euler_step gives them, and the score bit for bit the oracle's float32
+    L1 relative change of the updated (v_hat_prev, v_hat); a third of the tokens
+    are active, the rest score from caches they did not touch this step."""
+    need_gpu()
+    ctx, counts = _ctx(N, [40, 20, 10])
+    r = synth.rng(N + 7)
+    x, vh, vp, vf = (r.standard_normal((N, 16), dtype=np.float32) for _ in range(4))
+    vp[::5] = vh[::5] + np.float32(0.01) * vp[::5]          # a low-change region
+    mask = (r.random(N) < 0.35).astype(np.uint8)
+    sig = O.sigma_schedule(40, 5.0)
+    i = 23
+    xd, vhd, vpd = dev(x), dev(vh), dev(vp)
+    score = torch.full((N,), -1.0, dtype=torch.float32, device="cuda")
+    abi.hsa_euler_step_score(ctx, xd, vhd, vpd, dev(vf), dev(mask), sig[i], sig[i + 1], score)
+    abi.hsa_sync_check(ctx)
+    ex, eh, ep = O.euler_step_f32(x, vh, vp, vf, mask, sig[i], sig[i + 1])
+    assert (host(xd).view(np.uint32) == ex.view(np.uint32)).all()
+    assert (host(vhd) == eh).all() and (host(vpd) == ep).all()
+    want = O.l1_relative_change(ep, eh)
+    assert (host(score).view(np.uint32) == want.view(np.uint32)).all()
+    # the same buffer through the standalone score kernel
+    s2 = torch.empty((N,), dtype=torch.float32, device="cuda")
+    abi.hsa_score(ctx, vpd, vhd, s2)
+    assert (host(s2).view(np.uint32) == want.view(np.uint32)).all()
+    ctx.close()
+
+
 def test_euler_all_skipped_and_closed_form():
     """Mask all zero: caches untouched; T steps telescope to x0 + v (sigma_T - sigma_0)."""
     need_gpu()

@@ -18,10 +18,10 @@ LIB_PATH = os.path.join(PKG, "libhsa.so")
 # Every symbol the header declares, in header order.
 SYMBOLS = [
     "hsa_create", "hsa_destroy", "hsa_last_error", "hsa_set_stream", "hsa_sync_check",
-    "hsa_selftest_timeout", "hsa_kernel_launches", "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
+    "hsa_selftest_timeout", "hsa_kernel_launches", "hsa_time_kernels", "hsa_kernel_times", "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
     "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_linear", "hsa_kv_scatter", "hsa_kv_scatter_packed",
     "hsa_attention", "hsa_attention_kv", "hsa_out_proj_residual", "hsa_mlp_residual",
-    "hsa_layer_forward", "hsa_layer_forward_cond", "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_step", "hsa_step_cond",
+    "hsa_layer_forward", "hsa_layer_forward_cond", "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_euler_step_score", "hsa_step", "hsa_step_cond",
     "hsa_select_groups_static",
 ]
 
@@ -62,6 +62,13 @@ class hsa_model_weights(ctypes.Structure):
                 ("layers", ctypes.POINTER(hsa_layer_weights))]
 
 
+class hsa_kernel_class_time(ctypes.Structure):
+    _fields_ = [("calls", ctypes.c_uint64), ("ms", ctypes.c_double), ("work", ctypes.c_double)]
+
+
+KERNEL_CLASSES = ("attention", "gemm", "rows", "tokens")
+
+
 class hsa_state(ctypes.Structure):
     _fields_ = [("x", ctypes.c_void_p), ("v_hat", ctypes.c_void_p),
                 ("v_hat_prev", ctypes.c_void_p), ("v_fresh", ctypes.c_void_p),
@@ -93,6 +100,8 @@ def load() -> ctypes.CDLL:
         "hsa_sync_check": (I, [P]),
         "hsa_selftest_timeout": (I, [P, I]),
         "hsa_kernel_launches": (ctypes.c_uint64, [P]),
+        "hsa_time_kernels": (I, [P, I]),
+        "hsa_kernel_times": (I, [P, ctypes.POINTER(hsa_kernel_class_time), I]),
         "hsa_n_active": (I, [P, I]),
         "hsa_schedule": (I, [P, I, P, P, P, P, ctypes.POINTER(I)]),
         "hsa_score": (I, [P, P, P, P]),
@@ -113,6 +122,7 @@ def load() -> ctypes.CDLL:
         "hsa_embed": (I, [P, P, P, P, I, P]),
         "hsa_head": (I, [P, P, P, P, I, P]),
         "hsa_euler_step": (I, [P, P, P, P, P, P, F, F]),
+        "hsa_euler_step_score": (I, [P, P, P, P, P, P, F, F, P]),
         "hsa_step": (I, [P, ctypes.POINTER(hsa_model_weights), ctypes.POINTER(hsa_state), I, F, F, I]),
         "hsa_step_cond": (I, [P, ctypes.POINTER(hsa_model_weights), ctypes.POINTER(hsa_state),
                               ctypes.POINTER(hsa_cond), I, F, F, I]),
@@ -200,6 +210,20 @@ def hsa_selftest_timeout(ctx: Context, timeout_us: int) -> None:
 
 def hsa_kernel_launches(ctx: Context) -> int:
     return int(load().hsa_kernel_launches(ctx.ptr))
+
+
+def hsa_time_kernels(ctx: Context, on: bool) -> None:
+    _check(ctx.ptr, load().hsa_time_kernels(ctx.ptr, 1 if on else 0))
+
+
+def hsa_kernel_times(ctx: Context) -> dict:
+    """Per-class totals since timing was turned on or last read: {class:
+    {"calls", "ms", "work"}} (work: FLOP for attention and GEMM, bytes for row
+    kernels); reading clears them."""
+    out = (hsa_kernel_class_time * len(KERNEL_CLASSES))()
+    _check(ctx.ptr, load().hsa_kernel_times(ctx.ptr, out, len(KERNEL_CLASSES)))
+    return {name: {"calls": int(out[k].calls), "ms": float(out[k].ms), "work": float(out[k].work)}
+            for k, name in enumerate(KERNEL_CLASSES)}
 
 
 def hsa_n_active(ctx: Context, i: int) -> int:
@@ -304,6 +328,13 @@ def hsa_euler_step(ctx: Context, x, v_hat, v_hat_prev, v_fresh, mask, sigma_i: f
                    sigma_next: float) -> None:
     _check(ctx.ptr, load().hsa_euler_step(ctx.ptr, _p(x), _p(v_hat), _p(v_hat_prev), _p(v_fresh),
                                           _p(mask), float(sigma_i), float(sigma_next)))
+
+
+def hsa_euler_step_score(ctx: Context, x, v_hat, v_hat_prev, v_fresh, mask, sigma_i: float,
+                         sigma_next: float, score) -> None:
+    _check(ctx.ptr, load().hsa_euler_step_score(ctx.ptr, _p(x), _p(v_hat), _p(v_hat_prev),
+                                                _p(v_fresh), _p(mask), float(sigma_i),
+                                                float(sigma_next), _p(score)))
 
 
 class ModelBinding:

@@ -185,6 +185,9 @@ void hsa_destroy(hsa_ctx* ctx) {
   if (ctx == nullptr) return;
   Ctx& x = ctx->c;
   cudaStreamSynchronize(x.stream);
+  for (auto& r : x.times)
+    for (cudaEvent_t ev : r.pairs) cudaEventDestroy(ev);
+  for (cudaEvent_t ev : x.event_pool) cudaEventDestroy(ev);
   cudaFree(x.u);
   cudaFree(x.q);
   cudaFree(x.o);
@@ -228,6 +231,39 @@ hsa_status hsa_selftest_timeout(hsa_ctx* ctx, int timeout_us) {
 }
 
 uint64_t hsa_kernel_launches(const hsa_ctx* ctx) { return ctx ? ctx->c.launches : 0; }
+
+hsa_status hsa_time_kernels(hsa_ctx* ctx, int on) {
+  HSA_CHECK_CTX(ctx);
+  ctx->c.timing = on != 0;
+  return HSA_OK;
+}
+
+hsa_status hsa_kernel_times(hsa_ctx* ctx, hsa_kernel_class_time* out, int n_classes) {
+  HSA_CHECK_CTX(ctx);
+  if (out == nullptr || n_classes < 0) return fail(ctx, HSA_ERR_INVALID_ARG, "out is NULL");
+  Ctx& c = ctx->c;
+  cudaError_t e = cudaStreamSynchronize(c.stream);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "stream synchronize");
+  hsa_status st = HSA_OK;
+  for (int k = 0; k < hsa::TC_COUNT; ++k) {
+    hsa::TimeRec& r = c.times[k];
+    double ms = 0.0;
+    for (size_t j = 0; j + 1 < r.pairs.size(); j += 2) {
+      float t = 0.f;
+      e = cudaEventElapsedTime(&t, r.pairs[j], r.pairs[j + 1]);
+      if (e != cudaSuccess) st = cuda_fail(ctx, e, "event elapsed time");
+      ms += t;
+    }
+    if (k < n_classes) {
+      out[k].calls = r.calls;
+      out[k].ms = ms;
+      out[k].work = r.work;
+    }
+    for (cudaEvent_t ev : r.pairs) c.event_pool.push_back(ev);
+    r = hsa::TimeRec{};
+  }
+  return st;
+}
 
 int hsa_n_active(const hsa_ctx* ctx, int i) {
   if (ctx == nullptr || i < 0 || i >= ctx->c.T) return -1;
@@ -568,6 +604,21 @@ hsa_status hsa_euler_step(hsa_ctx* ctx, float* x, float* v_hat, float* v_hat_pre
                   "euler");
 }
 
+hsa_status hsa_euler_step_score(hsa_ctx* ctx, float* x, float* v_hat, float* v_hat_prev,
+                                const float* v_fresh, const uint8_t* mask, float sigma_i,
+                                float sigma_next, float* score) {
+  HSA_CHECK_CTX(ctx);
+  HSA_CHECK_PTR(ctx, x);
+  HSA_CHECK_PTR(ctx, v_hat);
+  HSA_CHECK_PTR(ctx, v_hat_prev);
+  HSA_CHECK_PTR(ctx, v_fresh);
+  HSA_CHECK_PTR(ctx, mask);
+  HSA_CHECK_PTR(ctx, score);
+  return launched(ctx, hsa::launch_euler(ctx->c, x, v_hat, v_hat_prev, v_fresh, mask, sigma_i,
+                                         sigma_next, score),
+                  "euler_score");
+}
+
 hsa_status hsa_step(hsa_ctx* ctx, const hsa_model_weights* w, const hsa_state* s, int i,
                     float sigma_i, float sigma_next, int regroup) {
   return hsa_step_cond(ctx, w, s, nullptr, i, sigma_i, sigma_next, regroup);
@@ -591,13 +642,17 @@ hsa_status hsa_step_cond(hsa_ctx* ctx, const hsa_model_weights* w, const hsa_sta
                                 s->k_cache[l], s->v_cache[l]);
   }
   if (st == HSA_OK) st = hsa_head(ctx, w->w_head, s->h, s->active_idx, n, s->v_fresh);
-  if (st == HSA_OK)
+  // re-grouping from iteration T / s_K on (every token then has two cached
+  // velocities), not after the last; its score is written by the Euler pass
+  const int from = ctx->c.T / ctx->c.budgets[ctx->c.K - 1];
+  const bool regroup_now = regroup && i >= from && i < ctx->c.T - 1;
+  if (st == HSA_OK && !regroup_now)
     st = hsa_euler_step(ctx, s->x, s->v_hat, s->v_hat_prev, s->v_fresh, s->mask, sigma_i,
                         sigma_next);
-  int smin = ctx->c.budgets[ctx->c.K - 1];
-  const int from = ctx->c.T / smin;
-  if (st == HSA_OK && regroup && i >= from && i < ctx->c.T - 1)
-    st = hsa_select_groups(ctx, s->v_hat_prev, s->v_hat, s->score, s->g);
+  if (st == HSA_OK && regroup_now)
+    st = hsa_euler_step_score(ctx, s->x, s->v_hat, s->v_hat_prev, s->v_fresh, s->mask, sigma_i,
+                              sigma_next, s->score);
+  if (st == HSA_OK && regroup_now) st = hsa_select_from_score(ctx, s->score, s->g);
   return st;
 }
 

@@ -7,6 +7,7 @@
 
 #include <atomic>
 #include <string>
+#include <vector>
 
 #include "../../include/hsa.h"
 
@@ -23,6 +24,15 @@ constexpr int kRadixBins = 256;
 // kMaxAttnParts x 256 rows x 128 fp32 = 64 MiB).
 constexpr int kMaxSplitParts = 32;
 constexpr int kMaxAttnParts = 512;
+
+// Kernel classes timed by hsa_time_kernels (CUDA events around each launch).
+enum TimeClass : int { TC_ATTN = 0, TC_GEMM = 1, TC_ROWS = 2, TC_TOKENS = 3, TC_COUNT = 4 };
+
+struct TimeRec {
+  std::vector<cudaEvent_t> pairs;  // start, stop, start, stop, ...
+  uint64_t calls = 0;
+  double work = 0.0;  // algorithmic FLOP (attention, GEMM) or bytes (rows, tokens)
+};
 
 struct Ctx {
   hsa_model_cfg cfg{};
@@ -44,6 +54,48 @@ struct Ctx {
   float* attn_part_ml = nullptr;  // [kMaxAttnParts][256][2] partial (max, sum)
   uint32_t* cuts = nullptr;  // selector cut keys, 2 words per cut
   int* flag = nullptr;       // device error flag
+  // per-launch timing (off unless hsa_time_kernels turned it on)
+  mutable bool timing = false;
+  mutable TimeRec times[TC_COUNT];
+  mutable std::vector<cudaEvent_t> event_pool;
+  cudaEvent_t take_event() const {
+    cudaEvent_t e = nullptr;
+    if (!event_pool.empty()) {
+      e = event_pool.back();
+      event_pool.pop_back();
+    } else if (cudaEventCreate(&e) != cudaSuccess) {
+      e = nullptr;
+    }
+    return e;
+  }
+};
+
+// While timing is on, brackets the launches made in its scope with two CUDA
+// events on the context's stream and adds `work` to the class's total.
+class Timed {
+ public:
+  Timed(const Ctx& c, int cls, double work) : c_(c), cls_(cls) {
+    if (!c_.timing) return;
+    start_ = c_.take_event();
+    if (start_ != nullptr) cudaEventRecord(start_, c_.stream);
+    c_.times[cls_].work += work;
+    c_.times[cls_].calls += 1;
+  }
+  ~Timed() {
+    if (!c_.timing || start_ == nullptr) return;
+    cudaEvent_t stop = c_.take_event();
+    if (stop == nullptr) return;
+    cudaEventRecord(stop, c_.stream);
+    c_.times[cls_].pairs.push_back(start_);
+    c_.times[cls_].pairs.push_back(stop);
+  }
+  Timed(const Timed&) = delete;
+  Timed& operator=(const Timed&) = delete;
+
+ private:
+  const Ctx& c_;
+  int cls_;
+  cudaEvent_t start_ = nullptr;
 };
 
 // Row-index guard used by kernels that follow idx: out-of-range rows are
@@ -74,8 +126,11 @@ cudaError_t launch_select_groups_raw(cudaStream_t stream, const float* v_prev, c
                                      int N, const int* counts, int K, float* score,
                                      uint32_t* cuts, uint8_t* g, int* flag);
 cudaError_t launch_selftest_timeout(const Ctx& c, uint64_t limit_ns);
+// With `score` set, the same pass also writes the re-grouping score of every
+// token from the updated (v_hat_prev, v_hat), bit for bit as launch_score does.
 cudaError_t launch_euler(const Ctx& c, float* x, float* v_hat, float* v_hat_prev,
-                         const float* v_fresh, const uint8_t* mask, float s0, float s1);
+                         const float* v_fresh, const uint8_t* mask, float s0, float s1,
+                         float* score = nullptr);
 cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, int n, void* u,
                              const float* shift = nullptr, const float* scale = nullptr);
 cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_rows, int src_ld,

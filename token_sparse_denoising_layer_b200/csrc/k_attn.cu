@@ -453,6 +453,7 @@ cudaError_t launch_hd(const Ctx& c, const void* q, int n, const void* kc, const 
 cudaError_t launch_attention(const Ctx& c, const void* q, int n, const void* kc, const void* vc,
                              int n_kv, void* o, std::string* why) {
   if (n <= 0) return cudaSuccess;
+  Timed timed(c, TC_ATTN, 4.0 * n * n_kv * c.cfg.D);
   const int d = c.cfg.D / c.cfg.H;
   if (d == 128) return launch_hd<128>(c, q, n, kc, vc, n_kv, o, why);
   if (d == 64) return launch_hd<64>(c, q, n, kc, vc, n_kv, o, why);

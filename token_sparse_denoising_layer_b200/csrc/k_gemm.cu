@@ -517,6 +517,7 @@ cudaError_t launch_bn(const Ctx& c, const GemmArgs& a, std::string* why) {
 
 cudaError_t launch_gemm(const Ctx& c, const GemmArgs& a, std::string* why) {
   if (a.M <= 0) return cudaSuccess;
+  Timed timed(c, TC_GEMM, 2.0 * a.M * a.Ncols * a.Kd);
   if (a.Kd % kBK != 0 || a.Ncols % 32 != 0) {
     if (why) *why = "GEMM needs K % 64 == 0 and Ncols % 32 == 0";
     return cudaErrorInvalidValue;

@@ -132,6 +132,7 @@ cudaError_t launch_ln_gather(const Ctx& c, const float* x, const int32_t* idx, i
                              const float* shift, const float* scale) {
   if (n <= 0) return cudaSuccess;
   const int D = c.cfg.D, N = c.cfg.N;
+  Timed timed(c, TC_ROWS, static_cast<double>(n) * D * (4 + 2));
   const dim3 grid((n + 7) / 8), block(256);
   auto* uo = static_cast<__nv_bfloat16*>(u);
   switch (D / 128) {
@@ -172,6 +173,7 @@ __global__ void __launch_bounds__(256) k_kv_scatter(const uint4* __restrict__ k_
 cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_rows, int src_ld,
                               const int32_t* idx, int n, void* kc, void* vc) {
   if (n <= 0) return cudaSuccess;
+  Timed timed(c, TC_ROWS, static_cast<double>(n) * c.cfg.D * 2 * 2 * 2);
   const int vpr = c.cfg.D / 8;
   const size_t total = static_cast<size_t>(n) * vpr;
   size_t blocks = (total + 255) / 256;
@@ -230,6 +232,7 @@ __global__ void __launch_bounds__(256) k_embed(const float* __restrict__ w_in,
 cudaError_t launch_embed(const Ctx& c, const float* w_in, const float* x_lat, const int32_t* idx,
                          int n, float* h) {
   if (n <= 0) return cudaSuccess;
+  Timed timed(c, TC_ROWS, static_cast<double>(n) * (64 + 4.0 * c.cfg.D));
   const size_t total = static_cast<size_t>(n) * (c.cfg.D / 4);
   k_embed<<<static_cast<unsigned>((total + 255) / 256), 256, 0, c.stream>>>(
       w_in, x_lat, idx, n, c.cfg.N, c.cfg.D, h, c.flag);
@@ -294,6 +297,7 @@ __global__ void __launch_bounds__(256) k_head(const float* __restrict__ w_head,
 cudaError_t launch_head(const Ctx& c, const float* w_head, const float* h, const int32_t* idx,
                         int n, float* v_fresh) {
   if (n <= 0) return cudaSuccess;
+  Timed timed(c, TC_ROWS, static_cast<double>(n) * (4.0 * c.cfg.D + 64));
   k_head<<<(n + 7) / 8, 256, 0, c.stream>>>(w_head, h, idx, n, c.cfg.N, c.cfg.D, v_fresh, c.flag);
   c.launches += 1;
   return cudaGetLastError();

@@ -14,6 +14,7 @@
 // call's contents; calls that overlap on the GPU (on two streams, or from two
 // threads) race on it.
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -35,21 +36,55 @@ static __device__ __align__(256) unsigned char g_select_scratch[kScratchBytes];
 constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void* g_scratch_addr[kMaxDevices] = {};
+unsigned long long g_scratch_ctx[kMaxDevices] = {};  // id of the context the address is for
 
-// Device address of the scratch array on the current device, looked up once
-// per device.  In host code the array's name is only a host-side stand-in.
-// Errors are reported by status code only: this entry point has no context to
-// hold a message.
+// Unique id of the current CUDA context (cuCtxGetId, through the runtime's
+// driver entry point), or 0 when the driver cannot say.
+unsigned long long current_context_id() {
+  typedef CUresult (*GetCurrentFn)(CUcontext*);
+  typedef CUresult (*GetIdFn)(CUcontext, unsigned long long*);
+  static GetCurrentFn get_current = nullptr;
+  static GetIdFn get_id = nullptr;
+  static bool looked = false;
+  if (!looked) {
+    void* a = nullptr;
+    void* b = nullptr;
+    cudaDriverEntryPointQueryResult qa, qb;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &a, cudaEnableDefault, &qa) == cudaSuccess &&
+        qa == cudaDriverEntryPointSuccess &&
+        cudaGetDriverEntryPoint("cuCtxGetId", &b, cudaEnableDefault, &qb) == cudaSuccess &&
+        qb == cudaDriverEntryPointSuccess) {
+      get_current = reinterpret_cast<GetCurrentFn>(a);
+      get_id = reinterpret_cast<GetIdFn>(b);
+    }
+    looked = true;
+  }
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != CUDA_SUCCESS ||
+      ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device.  In host code
+// the array's name is only a host-side stand-in.  The address is looked up
+// once per device and context: the first call on a device does it, and so
+// does the first call after a device reset replaced the context (or every
+// call, if the context cannot be identified).  Errors are reported by status
+// code only: this entry point has no context to hold a message.
 hsa_status scratch_address(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return HSA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return HSA_ERR_INVALID_ARG;
   std::lock_guard<std::mutex> lock(g_setup_mutex);
-  if (g_scratch_addr[dev] == nullptr) {
+  const unsigned long long ctx_id = current_context_id();
+  if (g_scratch_addr[dev] == nullptr || ctx_id == 0 || ctx_id != g_scratch_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_select_scratch) != cudaSuccess || p == nullptr)
       return HSA_ERR_CUDA;
     g_scratch_addr[dev] = p;
+    g_scratch_ctx[dev] = ctx_id;
   }
   *out = g_scratch_addr[dev];
   return HSA_OK;

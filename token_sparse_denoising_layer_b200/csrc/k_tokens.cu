@@ -18,11 +18,14 @@ namespace hsa {
 //
 // Token n of group k is active at iteration i iff i mod (T/s_k) == 0; in the
 // phase window (first/last m iterations, section 2.4) every token is active.
-// Each CTA owns a 4096-token chunk.  It counts the active tokens of all
-// earlier chunks itself (a read of at most N bytes from L2), so the compaction
-// needs one launch and no inter-CTA waiting.  Output order is ascending.
+// Each CTA owns a 1024-token chunk (four tokens per thread, one 32-bit load
+// of group ids and one 32-bit mask store), so N = 32760 spreads over 32 CTAs
+// and N = 75600 over 74.  A CTA counts the active tokens of all earlier chunks
+// itself (at most N bytes, read from L2 with 16-byte loads), so the
+// compaction needs one launch and no inter-CTA waiting.  Output order is
+// ascending.
 
-constexpr int kSchedThreads = 1024;
+constexpr int kSchedThreads = 256;
 constexpr int kSchedChunk = kSchedThreads * 4;
 
 struct SchedParams {
@@ -91,46 +94,57 @@ __global__ void __launch_bounds__(kSchedThreads) k_schedule(const uint8_t* __res
   const uint32_t bits = active_group_bits(p);
   const int base = blockIdx.x * kSchedChunk;
 
-  // 1. active tokens before this chunk (base is a multiple of 16)
+  // 1. this thread's four tokens (g and mask are 16-byte aligned, base and n0
+  //    are multiples of 4: a whole word is in bounds unless it holds the tail)
+  const int n0 = base + 4 * threadIdx.x;
+  uint32_t gw = 0xFFFFFFFFu;
+  if (n0 + 4 <= p.N) {
+    gw = __ldg(reinterpret_cast<const uint32_t*>(g + n0));
+  } else {
+    for (int j = 0; j < 4 && n0 + j < p.N; ++j)
+      gw = (gw & ~(0xFFu << (8 * j))) | (static_cast<uint32_t>(g[n0 + j]) << (8 * j));
+  }
+  int on[4];
+  int bad = 0;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const uint32_t gb = (gw >> (8 * j)) & 0xFFu;
+    const bool in = n0 + j < p.N;
+    if (in && gb >= static_cast<uint32_t>(p.K)) bad = 1;
+    on[j] = (in && gb < static_cast<uint32_t>(p.K)) ? on_of(gb, bits) : 0;
+  }
+  if (bad) atomicOr(flag, DEV_BAD_GROUP);
+
+  // 2. active tokens before this chunk (base is a multiple of 16)
   int before = 0;
   const uint4* gv = reinterpret_cast<const uint4*>(g);
+#pragma unroll 4
   for (int v = threadIdx.x; v < base / 16; v += blockDim.x) {
     const uint4 w = __ldg(gv + v);
     before += count_on_word(w.x, bits) + count_on_word(w.y, bits) + count_on_word(w.z, bits) +
               count_on_word(w.w, bits);
   }
-  before = block_sum(before, warp_sums);
-
-  // 2. this thread's four tokens
-  const int n0 = base + 4 * threadIdx.x;
-  int on[4] = {0, 0, 0, 0};
-  int bad = 0;
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int n = n0 + j;
-    if (n < p.N) {
-      const uint32_t gb = g[n];
-      if (gb >= static_cast<uint32_t>(p.K)) bad = 1;
-      else on[j] = on_of(gb, bits);
-    }
-  }
-  if (bad) atomicOr(flag, DEV_BAD_GROUP);
   const int mine = on[0] + on[1] + on[2] + on[3];
+  before = block_sum(before, warp_sums);
   int total;
   int pos = before + block_exclusive_scan(mine, warp_sums, &total);
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const int n = n0 + j;
-    if (n < p.N) {
-      mask[n] = static_cast<uint8_t>(on[j]);
-      if (on[j]) idx[pos++] = n;
-    }
+  if (n0 + 4 <= p.N) {
+    *reinterpret_cast<uint32_t*>(mask + n0) = static_cast<uint32_t>(on[0]) |
+                                              (static_cast<uint32_t>(on[1]) << 8) |
+                                              (static_cast<uint32_t>(on[2]) << 16) |
+                                              (static_cast<uint32_t>(on[3]) << 24);
+  } else {
+    for (int j = 0; j < 4 && n0 + j < p.N; ++j) mask[n0 + j] = static_cast<uint8_t>(on[j]);
   }
+#pragma unroll
+  for (int j = 0; j < 4; ++j)
+    if (on[j]) idx[pos++] = n0 + j;
   if (n_dev != nullptr && threadIdx.x == 0 && base + kSchedChunk >= p.N) *n_dev = before + total;
 }
 
 cudaError_t launch_schedule(const Ctx& c, int i, const uint8_t* g, uint8_t* mask, int32_t* idx,
                             int32_t* n_dev) {
+  Timed timed(c, TC_TOKENS, 0.0);
   SchedParams p{};
   for (int k = 0; k < c.K; ++k) p.strides[k] = c.strides[k];
   p.K = c.K;
@@ -178,6 +192,7 @@ __global__ void __launch_bounds__(256) k_score(const float4* __restrict__ v_prev
 }
 
 cudaError_t launch_score(const Ctx& c, const float* v_prev, const float* v_cur, float* score) {
+  Timed timed(c, TC_TOKENS, 0.0);
   const int N = c.cfg.N;
   k_score<<<(N + 255) / 256, 256, 0, c.stream>>>(reinterpret_cast<const float4*>(v_prev),
                                                  reinterpret_cast<const float4*>(v_cur), score, N,
@@ -428,6 +443,7 @@ __global__ void __launch_bounds__(256) k_assign(const float* __restrict__ score,
 }
 
 cudaError_t launch_select(const Ctx& c, const float* score, uint8_t* g) {
+  Timed timed(c, TC_TOKENS, 0.0);
   const int N = c.cfg.N;
   const int ncut = c.K - 1;
   if (ncut == 0) {
@@ -510,38 +526,98 @@ cudaError_t launch_selftest_timeout(const Ctx& c, uint64_t limit_ns) {
 // then every token advances by (sigma_next - sigma_i) * v_hat.  Inactive
 // tokens read neither v_fresh nor write the caches (predicated, not branched
 // per warp).  Float32 with one rounding per operation.
+//
+// With kScore the same pass also writes the re-grouping score of every token
+// from the two caches as they leave it (section 2.1, Dynamic Selection), so a
+// re-grouping step reads the velocities once: the four threads of a token
+// hold channels 0-3, 4-7, 8-11, 12-15, and the two sums run through them in
+// channel order (each thread continues its left neighbour's partial sums), in
+// the same order and rounding as k_score.
 
+template <bool kScore>
 __global__ void __launch_bounds__(256) k_euler(float4* __restrict__ x, float4* __restrict__ v_hat,
                                                float4* __restrict__ v_hat_prev,
                                                const float4* __restrict__ v_fresh,
                                                const uint8_t* __restrict__ mask, float s0,
-                                               float s1, int n4) {
+                                               float s1, int n4, float* __restrict__ score,
+                                               int* flag) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= n4) return;
+  if (!kScore && t >= n4) return;
+  const bool live = t < n4;  // n4 = 4N: a token's four threads are all live or all not
   const float d = __fsub_rn(s1, s0);
-  const bool on = __ldg(mask + (t >> 2)) != 0;
-  float4 h = __ldcs(v_hat + t);
-  float4 xx = __ldcs(x + t);
+  const bool on = live && __ldg(mask + (t >> 2)) != 0;
+  float4 h = make_float4(0.f, 0.f, 0.f, 0.f), xx = h, prev = h;
+  if (live) {
+    h = kScore ? v_hat[t] : __ldcs(v_hat + t);
+    xx = __ldcs(x + t);
+  }
   if (on) {
     const float4 f = __ldcs(v_fresh + t);
-    __stcs(v_hat_prev + t, h);
-    __stcs(v_hat + t, f);
+    if (kScore) {
+      v_hat_prev[t] = h;
+      v_hat[t] = f;
+    } else {
+      __stcs(v_hat_prev + t, h);
+      __stcs(v_hat + t, f);
+    }
+    prev = h;
     h = f;
+  } else if (kScore && live) {
+    prev = v_hat_prev[t];
   }
-  xx.x = __fadd_rn(xx.x, __fmul_rn(d, h.x));
-  xx.y = __fadd_rn(xx.y, __fmul_rn(d, h.y));
-  xx.z = __fadd_rn(xx.z, __fmul_rn(d, h.z));
-  xx.w = __fadd_rn(xx.w, __fmul_rn(d, h.w));
-  __stcs(x + t, xx);
+  if (live) {
+    xx.x = __fadd_rn(xx.x, __fmul_rn(d, h.x));
+    xx.y = __fadd_rn(xx.y, __fmul_rn(d, h.y));
+    xx.z = __fadd_rn(xx.z, __fmul_rn(d, h.z));
+    xx.w = __fadd_rn(xx.w, __fmul_rn(d, h.w));
+    __stcs(x + t, xx);
+  }
+  if (kScore) {
+    const int q = threadIdx.x & 3;  // blockDim is a multiple of 4: quads stay in one warp
+    float num = 0.f, den = 0.f;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float pn = __shfl_up_sync(0xffffffffu, num, 1);
+      const float pd = __shfl_up_sync(0xffffffffu, den, 1);
+      if (q == r) {
+        float a = r == 0 ? 0.f : pn, b = r == 0 ? 0.f : pd;
+        a = __fadd_rn(a, fabsf(__fsub_rn(h.x, prev.x)));
+        b = __fadd_rn(b, fabsf(prev.x));
+        a = __fadd_rn(a, fabsf(__fsub_rn(h.y, prev.y)));
+        b = __fadd_rn(b, fabsf(prev.y));
+        a = __fadd_rn(a, fabsf(__fsub_rn(h.z, prev.z)));
+        b = __fadd_rn(b, fabsf(prev.z));
+        a = __fadd_rn(a, fabsf(__fsub_rn(h.w, prev.w)));
+        b = __fadd_rn(b, fabsf(prev.w));
+        num = a;
+        den = b;
+      }
+    }
+    if (q == 3 && live) {
+      den = __fadd_rn(den, kScoreEps);
+      const float r = __fadd_rn(__fdiv_rn(num, den), 0.0f);
+      if (!(r >= 0.f) || isinf(r)) atomicOr(flag, DEV_BAD_SCORE);
+      score[t >> 2] = r;
+    }
+  }
 }
 
 cudaError_t launch_euler(const Ctx& c, float* x, float* v_hat, float* v_hat_prev,
-                         const float* v_fresh, const uint8_t* mask, float s0, float s1) {
+                         const float* v_fresh, const uint8_t* mask, float s0, float s1,
+                         float* score) {
+  Timed timed(c, TC_TOKENS, 0.0);
   const int n4 = c.cfg.N * (c.cfg.C / 4);
-  k_euler<<<(n4 + 255) / 256, 256, 0, c.stream>>>(
-      reinterpret_cast<float4*>(x), reinterpret_cast<float4*>(v_hat),
-      reinterpret_cast<float4*>(v_hat_prev), reinterpret_cast<const float4*>(v_fresh), mask, s0,
-      s1, n4);
+  const dim3 grid((n4 + 255) / 256);
+  if (score != nullptr)
+    k_euler<true><<<grid, 256, 0, c.stream>>>(
+        reinterpret_cast<float4*>(x), reinterpret_cast<float4*>(v_hat),
+        reinterpret_cast<float4*>(v_hat_prev), reinterpret_cast<const float4*>(v_fresh), mask,
+        s0, s1, n4, score, c.flag);
+  else
+    k_euler<false><<<grid, 256, 0, c.stream>>>(
+        reinterpret_cast<float4*>(x), reinterpret_cast<float4*>(v_hat),
+        reinterpret_cast<float4*>(v_hat_prev), reinterpret_cast<const float4*>(v_fresh), mask,
+        s0, s1, n4, nullptr, c.flag);
   c.launches += 1;
   return cudaGetLastError();
 }
