@@ -203,3 +203,74 @@ def test_layer_stages(N, D, H, F, a):
     print(errs)
     abi.hsa_sync_check(ctx)
     assert all(e <= BF16_TOL for e in errs.values()), errs
+
+
+def _bf16_ulp(v):
+    """Spacing of bf16 values at |v| (8 significant bits)."""
+    e = np.floor(np.log2(np.maximum(np.abs(v), 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+def test_gelu_epilogue_within_bf16_rounding_of_exact_erf():
+    """The MLP's GELU epilogue computes erfc with a published Chebyshev fit
+    (Numerical Recipes section 6.2, fractional error < 1.2e-7).  With
+    W_1 = W_2 = I the residual update of each active row is exactly the stored
+    bf16 GELU of its LN output, so it is compared, value by value, with the
+    exact erf GELU (scipy, float64) of the same bf16 LN output: equal to its
+    bf16 rounding, or one bf16 step away where the exact value sits within
+    the approximation's error of a rounding boundary."""
+    need_gpu()
+    N, D, F, a = 4096, 128, 128, 4000
+    ctx = _ctx(N, D, 1, F)
+    r = synth.rng(77)
+    # small rows: x + GELU(u) then rounds far below GELU's bf16 step, so the
+    # update is recovered exactly (LN makes the scale irrelevant to u)
+    x = (r.standard_normal((N, D), dtype=np.float32) * np.float32(0.01)).astype(np.float32)
+    idx = synth.random_active_set(N, a, 77)
+    eye = torch.eye(D, dtype=torch.bfloat16, device="cuda")
+    xd, idd = dev(x), dev(idx)
+    u = torch.empty((a, D), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_ln_gather(ctx, xd, idd, a, u)
+    abi.hsa_mlp_residual(ctx, eye, eye, xd, idd, a)
+    abi.hsa_sync_check(ctx)
+    got = O.bf16(host(xd)[idx].astype(np.float64) - x[idx].astype(np.float64))
+    exact = O.gelu(host(u).astype(np.float64))
+    want = O.bf16(exact)
+    ulp = _bf16_ulp(want)
+    diff = np.abs(got - want)
+    assert (diff <= ulp * 1.0001).all()
+    assert (diff == 0).mean() >= 0.999
+
+
+@pytest.mark.parametrize("N,D,a", [(1, 128, 1), (300, 128, 17), (4096, 1536, 1000),
+                                   (32760, 1536, 32760), (2000, 5120, 333)])
+def test_embed_and_head(N, D, a):
+    """Latent embed of the active rows and the velocity head on them, fp32
+    kernels against the oracle's (pinned) embed and head, within 1e-5; rows
+    outside the active set are left untouched."""
+    need_gpu()
+    ctx = _ctx(N, D, D // 128, 64)
+    r = synth.rng(N + D + a)
+    w_in = (r.standard_normal((D, 16), dtype=np.float32) * np.float32(0.25)).astype(np.float32)
+    w_head = (r.standard_normal((16, D), dtype=np.float32) / np.float32(np.sqrt(D))).astype(np.float32)
+    x_lat = r.standard_normal((N, 16), dtype=np.float32)
+    idx = synth.random_active_set(N, a, N + 1)
+    h0 = r.standard_normal((N, D), dtype=np.float32)
+    hd = dev(h0)
+    abi.hsa_embed(ctx, dev(w_in), dev(x_lat), dev(idx), a, hd)
+    abi.hsa_sync_check(ctx)
+    hg = host(hd)
+    assert normwise(hg[idx], O.embed(w_in, x_lat[idx])) <= 1e-5
+    rest = np.setdiff1d(np.arange(N), idx)
+    assert (hg[rest] == h0[rest]).all()
+    # the head on the embedded rows (plus noise, so the LN is not degenerate)
+    hh = hg.copy()
+    hh[idx] += r.standard_normal((a, D), dtype=np.float32)
+    vf0 = np.full((N, 16), 7.0, dtype=np.float32)
+    vfd = dev(vf0)
+    abi.hsa_head(ctx, dev(w_head), dev(hh), dev(idx), a, vfd)
+    abi.hsa_sync_check(ctx)
+    vg = host(vfd)
+    assert normwise(vg[idx], O.head(w_head, hh[idx])) <= 1e-5
+    assert (vg[rest] == 7.0).all()
+    ctx.close()

@@ -9,11 +9,11 @@
 // and out-projection / MLP results are added into residual rows idx[m].
 //
 // Persistent: one CTA per SM walks its share of the 128 x BN output tiles
-// (BN = 256 or 128), K-block 64, through a multi-stage TMA ring that runs on
-// across tiles.  Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs (one
-// thread) into one of two TMEM accumulators, warps 2..5 drain the other
-// accumulator and run the epilogue, so a tile's epilogue overlaps the next
-// tile's main loop.
+// (BN = 256, 192 or 128), K-block 64, through a multi-stage TMA ring that runs
+// on across tiles.  Warp 0 issues TMA, warp 1 owns TMEM and issues the MMAs
+// (one thread) into one of two TMEM accumulators, and eight epilogue warps
+// drain the other accumulator (two per TMEM lane quarter, one per column
+// half), so a tile's epilogue overlaps the next tile's main loop.
 
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -31,20 +31,28 @@ namespace {
 
 constexpr int kBM = 128;
 constexpr int kBK = 64;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 320;  // TMA warp, MMA warp, 8 epilogue warps
+constexpr int kEpiWarps = 8;
 // relative cost per output element of a CTA-pair tile vs a 1-CTA 256-wide tile
 constexpr double kPairCost = 0.8;
 
+// Shared-memory staging for the residual epilogue: one 32 x 32 fp32 chunk
+// per epilogue warp.  The 16-byte group g of row r is stored at group
+// g ^ (r & 7), which keeps both the row-wise writes and the column-wise reads
+// below free of bank conflicts without padding.
+constexpr int kStageWarpFloats = 32 * 32;
+constexpr int kEpiStageBytes = kEpiWarps * kStageWarpFloats * 4;
+
 template <int BN>
 struct GemmCfg {
-  static constexpr int kStages = BN == 256 ? 4 : BN == 192 ? 5 : 6;
+  static constexpr int kStages = BN == 128 ? 6 : 4;
   // two accumulators of BN fp32 columns, allocated as a power of two
   static constexpr uint32_t kTmemCols = 2 * BN <= 256 ? 256 : 512;
   static constexpr int kABytes = kBM * kBK * 2;
   static constexpr int kBBytes = BN * kBK * 2;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kBarBytes = 256;
-  static constexpr int kSmem = kStages * kStageBytes + kBarBytes + 1024;
+  static constexpr int kSmem = kStages * kStageBytes + kBarBytes + kEpiStageBytes + 1024;
 };
 
 struct EpiParams {
@@ -61,8 +69,67 @@ struct EpiParams {
   int* flag;
 };
 
-__device__ __forceinline__ float gelu_f(float v) {
-  return 0.5f * v * (1.0f + erff(v * 0.70710678118654752440f));
+struct F2 {
+  float x, y;
+};
+
+// d = a * b + c, two lanes per instruction (packed f32x2).
+__device__ __forceinline__ F2 fma_x2(F2 a, F2 b, F2 c) {
+  F2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+__device__ __forceinline__ F2 mul_x2(F2 a, F2 b) {
+  F2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+__device__ __forceinline__ F2 splat(float v) { return F2{v, v}; }
+
+__device__ __forceinline__ float rcp_approx(float x) {
+  float y;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
+// GELU, erf form, of two values: v Phi(v), with Phi(v) = 1 - erfc(v / sqrt 2) / 2
+// for v >= 0 and erfc(|v| / sqrt 2) / 2 for v < 0.  erfc(z), z >= 0, is the
+// Chebyshev fit of Press, Teukolsky, Vetterling & Flannery, Numerical Recipes,
+// section 6.2: t = 1 / (1 + z/2), erfc(z) = t exp(-z^2 + P(t)) with a degree-9
+// P, a fractional error below 1.2e-7 for every z.  A relative bound matters
+// here: for v < 0 the result is a small tail value that is then rounded to
+// bf16.  Evaluated on packed f32x2 lanes with P's coefficients negated (Horner
+// commutes with negation), and the 1/2 folded into the exponent; two MUFU
+// operations per value, no branches.
+__device__ __forceinline__ F2 gelu_x2(F2 v) {
+  const F2 zn = F2{fabsf(v.x) * -0.70710678118654752440f, fabsf(v.y) * -0.70710678118654752440f};
+  const F2 d = fma_x2(zn, splat(-0.5f), splat(1.0f));  // 1 + z/2
+  const F2 t = F2{rcp_approx(d.x), rcp_approx(d.y)};
+  F2 q = fma_x2(splat(-0.17087277f), t, splat(0.82215223f));  // -P(t) by Horner
+  q = fma_x2(q, t, splat(-1.48851587f));
+  q = fma_x2(q, t, splat(1.13520398f));
+  q = fma_x2(q, t, splat(-0.27886807f));
+  q = fma_x2(q, t, splat(0.18628806f));
+  q = fma_x2(q, t, splat(-0.09678418f));
+  q = fma_x2(q, t, splat(-0.37409196f));
+  q = fma_x2(q, t, splat(-1.00002368f));
+  q = fma_x2(q, t, splat(1.26551223f));
+  q = fma_x2(zn, zn, q);  // z^2 - P(t)
+  // log2 of erfc(z) / 2 / t: (P(t) - z^2) log2(e) - 1
+  const F2 s = fma_x2(q, splat(-1.4426950408889634f), splat(-1.0f));
+  const F2 he = mul_x2(t, F2{ex2_approx(s.x), ex2_approx(s.y)});  // erfc(z) / 2
+  const F2 phi = F2{v.x >= 0.f ? 1.0f - he.x : he.x, v.y >= 0.f ? 1.0f - he.y : he.y};
+  return mul_x2(v, phi);
 }
 
 // 32 fp32 accumulators -> 32 bf16 at dst (64 contiguous bytes, 16-byte aligned).
@@ -77,8 +144,9 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t
       float a = __uint_as_float(r[8 * v + 2 * e]);
       float b = __uint_as_float(r[8 * v + 2 * e + 1]);
       if (kGelu) {
-        a = gelu_f(a);
-        b = gelu_f(b);
+        const F2 g = gelu_x2(F2{a, b});
+        a = g.x;
+        b = g.y;
       }
       w[e] = pack_bf16(a, b);
     }
@@ -86,19 +154,104 @@ __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const uint32_t
   }
 }
 
-// x[dst .. dst+31] += r, or += gate[..] * r with a gate (fp32, 128 contiguous bytes).
-__device__ __forceinline__ void add_f32x32(float* dst, const uint32_t (&r)[32], const float* gate) {
-  float4* d4 = reinterpret_cast<float4*>(dst);
+
+// x[dst_row(r), col .. col+31] += chunk row r for the warp's 32 rows, as
+// vector reductions that L2 performs, so the epilogue never waits for the
+// residual rows it updates.  The chunk (row r in lane r's registers) goes
+// through shared memory so that one reduction instruction covers four rows
+// and 128 contiguous bytes of each: lanes 8k'..8k'+7 own row 4k + k'.  Each
+// element gets exactly one addition per launch: x + v rounded once (with a
+// gate, gate * v is rounded first).
+__device__ __forceinline__ void resid_chunk(const EpiParams& p, const uint32_t (&r)[32],
+                                            int32_t dst_row, int col, float* stage) {
+  const int lane = threadIdx.x & 31;
+  float* srow = stage + lane * 32;
 #pragma unroll
-  for (int v = 0; v < 8; ++v) {
-    float4 a = d4[v];
-    float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
-    if (gate != nullptr) g = __ldg(reinterpret_cast<const float4*>(gate) + v);
-    a.x = fmaf(g.x, __uint_as_float(r[4 * v]), a.x);
-    a.y = fmaf(g.y, __uint_as_float(r[4 * v + 1]), a.y);
-    a.z = fmaf(g.z, __uint_as_float(r[4 * v + 2]), a.z);
-    a.w = fmaf(g.w, __uint_as_float(r[4 * v + 3]), a.w);
-    d4[v] = a;
+  for (int v = 0; v < 8; ++v)
+    *reinterpret_cast<float4*>(srow + 4 * (v ^ (lane & 7))) =
+        make_float4(__uint_as_float(r[4 * v]), __uint_as_float(r[4 * v + 1]),
+                    __uint_as_float(r[4 * v + 2]), __uint_as_float(r[4 * v + 3]));
+  __syncwarp();
+  const int g4 = lane & 7;  // this lane's 16-byte group of the row
+  float4 g = make_float4(1.f, 1.f, 1.f, 1.f);
+  if (p.gate != nullptr) g = __ldg(reinterpret_cast<const float4*>(p.gate + col + 4 * g4));
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const int rr = 4 * k + (lane >> 3);
+    const int32_t d = __shfl_sync(0xffffffffu, dst_row, rr);
+    float4 v = *reinterpret_cast<const float4*>(stage + rr * 32 + 4 * (g4 ^ (rr & 7)));
+    if (d >= 0) {
+      if (p.gate != nullptr) {
+        v.x *= g.x;
+        v.y *= g.y;
+        v.z *= g.z;
+        v.w *= g.w;
+      }
+      float* dst = p.x + static_cast<size_t>(d) * p.ld_x + col + 4 * g4;
+      asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(dst), "f"(v.x),
+                   "f"(v.y), "f"(v.z), "f"(v.w)
+                   : "memory");
+    }
+  }
+  __syncwarp();  // the stage is reused by the next chunk
+}
+
+// Drain one accumulator tile: this warp's 32 rows (TMEM lanes at tbase),
+// output row m (this lane's), columns n0 .. n0 + kCols - 1.  TMEM loads run
+// one 32-column chunk ahead of the chunk being stored.
+template <int kCols, int kEpi>
+__device__ __forceinline__ void drain_tile(const EpiParams& p, uint32_t tbase, int m, int n0,
+                                           float* stage) {
+  constexpr int NC = kCols / 32;
+  const bool mrow = m < p.M;
+  int32_t dst_row = -1;
+  if ((kEpi == EPI_QKV || kEpi == EPI_RESID) && mrow) {
+    dst_row = __ldg(p.idx + m);
+    if (!row_ok(dst_row, p.N, p.flag)) dst_row = -1;
+  }
+  uint32_t ra[32], rb[32];
+  __syncwarp();
+  tmem_ld32_nowait(tbase, ra);
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    uint32_t(&cur)[32] = (c & 1) ? rb : ra;
+    uint32_t(&nxt)[32] = (c & 1) ? ra : rb;
+    tmem_wait_ld();
+    if (c + 1 < NC) {
+      __syncwarp();
+      tmem_ld32_nowait(tbase + 32 * (c + 1), nxt);
+    }
+    const int col = n0 + 32 * c;
+    if (col >= p.Ncols) continue;  // uniform over the warp
+    if (kEpi == EPI_RESID) {
+      resid_chunk(p, cur, dst_row, col, stage);
+    } else if (mrow) {
+      if (kEpi == EPI_STORE || kEpi == EPI_GELU) {
+        store_bf16x32<kEpi == EPI_GELU>(p.out + static_cast<size_t>(m) * p.ld_out + col, cur);
+      } else {  // EPI_QKV
+        const int D = p.ld_out;
+        const int which = col / D;
+        const int cc = col - which * D;
+        if (which == 0) {
+          store_bf16x32<false>(p.out + static_cast<size_t>(m) * D + cc, cur);
+        } else if (dst_row >= 0) {
+          __nv_bfloat16* cache = which == 1 ? p.kc : p.vc;
+          store_bf16x32<false>(cache + static_cast<size_t>(dst_row) * D + cc, cur);
+        }
+      }
+    }
+  }
+}
+
+template <int kCols>
+__device__ __forceinline__ void drain(const EpiParams& p, uint32_t tbase, int m, int n0,
+                                      float* stage) {
+  switch (p.epi) {
+    case EPI_STORE: drain_tile<kCols, EPI_STORE>(p, tbase, m, n0, stage); break;
+    case EPI_GELU: drain_tile<kCols, EPI_GELU>(p, tbase, m, n0, stage); break;
+    case EPI_QKV: drain_tile<kCols, EPI_QKV>(p, tbase, m, n0, stage); break;
+    case EPI_RESID: drain_tile<kCols, EPI_RESID>(p, tbase, m, n0, stage); break;
+    default: break;
   }
 }
 
@@ -118,6 +271,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_full = empty + S;     // [2] accumulator buffer ready for the epilogue
   uint64_t* acc_empty = acc_full + 2; // [2] accumulator buffer drained
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  float* stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + Cfg::kBarBytes);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nk = p.Kd / kBK;
@@ -129,7 +283,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 4);  // one arrival per epilogue warp
+      mbar_init(&acc_empty[b], kEpiWarps);  // one arrival per epilogue warp
     }
     fence_barrier_init();
   }
@@ -203,8 +357,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else {
-    // epilogue: warp w reads TMEM lanes [32*(w%4), +32) = tile rows
+    // epilogue: warp w reads TMEM lanes [32*(w%4), +32) = tile rows, and
+    // column half (w - 2) / 4 of the tile
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int row = 32 * q + lane;
     int lt = 0;
     for (int t = blockIdx.x; t < total_tiles; t += gridDim.x, ++lt) {
@@ -214,48 +370,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m = (t / n_tiles) * kBM + row, n0 = (t % n_tiles) * BN;
-      const bool mrow = m < p.M;
-      int32_t dst_row = 0;
-      if (mrow && (p.epi == EPI_QKV || p.epi == EPI_RESID)) {
-        dst_row = __ldg(p.idx + m);
-        if (!row_ok(dst_row, p.N, p.flag)) dst_row = -1;
-      }
-      const uint32_t tbase = tmem + b * BN + (static_cast<uint32_t>(32 * q) << 16);
-#pragma unroll 1
-      for (int c0 = 0; c0 < BN; c0 += 32) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld32(tbase + c0, r);
-        const int col = n0 + c0;
-        if (mrow && col < p.Ncols) switch (p.epi) {
-          case EPI_STORE:
-            store_bf16x32<false>(p.out + static_cast<size_t>(m) * p.ld_out + col, r);
-            break;
-          case EPI_GELU:
-            store_bf16x32<true>(p.out + static_cast<size_t>(m) * p.ld_out + col, r);
-            break;
-          case EPI_QKV: {
-            const int D = p.ld_out;
-            const int which = col / D;
-            const int cc = col - which * D;
-            if (which == 0) {
-              store_bf16x32<false>(p.out + static_cast<size_t>(m) * D + cc, r);
-            } else if (dst_row >= 0) {
-              __nv_bfloat16* cache = which == 1 ? p.kc : p.vc;
-              store_bf16x32<false>(cache + static_cast<size_t>(dst_row) * D + cc, r);
-            }
-            break;
-          }
-          case EPI_RESID:
-            if (dst_row >= 0)
-              add_f32x32(p.x + static_cast<size_t>(dst_row) * p.ld_x + col, r,
-                         p.gate != nullptr ? p.gate + col : nullptr);
-            break;
-          default:
-            break;
-        }
-      }
+      const int m = (t / n_tiles) * kBM + row, n0 = (t % n_tiles) * BN + half * (BN / 2);
+      const uint32_t tbase =
+          tmem + b * BN + half * (BN / 2) + (static_cast<uint32_t>(32 * q) << 16);
+      drain<BN / 2>(p, tbase, m, n0, stage + (warp - 2) * kStageWarpFloats);
       // the buffer may be refilled once every lane's TMEM reads are done
       tc_fence_before();
       __syncwarp();
@@ -283,7 +401,7 @@ constexpr int kPairStages = 6;
 constexpr int kPairABytes = 128 * kBK * 2;
 constexpr int kPairBBytes = 128 * kBK * 2;
 constexpr int kPairStageBytes = kPairABytes + kPairBBytes;
-constexpr int kPairSmem = kPairStages * kPairStageBytes + 256 + 1024;
+constexpr int kPairSmem = kPairStages * kPairStageBytes + 256 + kEpiStageBytes + 1024;
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     k_gemm_pair(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
@@ -299,6 +417,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   uint64_t* acc_full = empty + S;      // [2]
   uint64_t* acc_empty = acc_full + 2;  // [2], used in rank 0
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+  float* stage = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + 256);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -312,7 +431,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 8);  // 4 epilogue warps in each CTA
+      mbar_init(&acc_empty[b], 2 * kEpiWarps);  // every epilogue warp of both CTAs
     }
     fence_barrier_init();
   }
@@ -380,6 +499,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     }
   } else {
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;  // column half of the tile
     const int row = 32 * q + lane;
     const uint32_t lead_empty0 = to_leader(smem_u32(&acc_empty[0]));
     const uint32_t lead_empty1 = to_leader(smem_u32(&acc_empty[1]));
@@ -391,48 +511,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
         break;
       }
       tc_fence_after();
-      const int m = (t / n_tiles) * 256 + rank * 128 + row, n0 = (t % n_tiles) * 256;
-      const bool mrow = m < p.M;
-      int32_t dst_row = 0;
-      if (mrow && (p.epi == EPI_QKV || p.epi == EPI_RESID)) {
-        dst_row = __ldg(p.idx + m);
-        if (!row_ok(dst_row, p.N, p.flag)) dst_row = -1;
-      }
-      const uint32_t tbase = tmem + b * 256 + (static_cast<uint32_t>(32 * q) << 16);
-#pragma unroll 1
-      for (int c0 = 0; c0 < 256; c0 += 32) {
-        uint32_t r[32];
-        __syncwarp();
-        tmem_ld32(tbase + c0, r);
-        const int col = n0 + c0;
-        if (mrow && col < p.Ncols) switch (p.epi) {
-          case EPI_STORE:
-            store_bf16x32<false>(p.out + static_cast<size_t>(m) * p.ld_out + col, r);
-            break;
-          case EPI_GELU:
-            store_bf16x32<true>(p.out + static_cast<size_t>(m) * p.ld_out + col, r);
-            break;
-          case EPI_QKV: {
-            const int D = p.ld_out;
-            const int which = col / D;
-            const int cc = col - which * D;
-            if (which == 0) {
-              store_bf16x32<false>(p.out + static_cast<size_t>(m) * D + cc, r);
-            } else if (dst_row >= 0) {
-              __nv_bfloat16* cache = which == 1 ? p.kc : p.vc;
-              store_bf16x32<false>(cache + static_cast<size_t>(dst_row) * D + cc, r);
-            }
-            break;
-          }
-          case EPI_RESID:
-            if (dst_row >= 0)
-              add_f32x32(p.x + static_cast<size_t>(dst_row) * p.ld_x + col, r,
-                         p.gate != nullptr ? p.gate + col : nullptr);
-            break;
-          default:
-            break;
-        }
-      }
+      const int m = (t / n_tiles) * 256 + rank * 128 + row, n0 = (t % n_tiles) * 256 + half * 128;
+      const uint32_t tbase = tmem + b * 256 + half * 128 + (static_cast<uint32_t>(32 * q) << 16);
+      drain<128>(p, tbase, m, n0, stage + (warp - 2) * kStageWarpFloats);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(b == 0 ? lead_empty0 : lead_empty1);
@@ -446,6 +527,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
     tmem_dealloc_pair(tmem, 512);
   }
 }
+
+static_assert(kPairSmem <= 227 * 1024, "CTA-pair GEMM exceeds the shared memory of a CTA");
+static_assert(GemmCfg<256>::kSmem <= 227 * 1024 && GemmCfg<192>::kSmem <= 227 * 1024 &&
+                  GemmCfg<128>::kSmem <= 227 * 1024,
+              "GEMM tile exceeds the shared memory of a CTA");
 
 cudaError_t launch_pair(const Ctx& c, const GemmArgs& a, std::string* why) {
   CUtensorMap ta, tb;

@@ -188,54 +188,73 @@ cudaError_t launch_kv_scatter(const Ctx& c, const void* k_rows, const void* v_ro
 }
 
 // ------------------------------------------------------------ embed
-// h[idx[m], j] = sum_c W_in[j, c] * x_lat[idx[m], c]; C = 16, four j per thread.
-__global__ void __launch_bounds__(256) k_embed(const float* __restrict__ w_in,
-                                               const float* __restrict__ x_lat,
-                                               const int32_t* __restrict__ idx, int n, int N,
-                                               int D, float* __restrict__ h, int* flag) {
-  const int q4 = D / 4;
-  const size_t t = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
-  if (t >= static_cast<size_t>(n) * q4) return;
-  const int m = static_cast<int>(t / q4);
-  const int j0 = static_cast<int>(t - static_cast<size_t>(m) * q4) * 4;
-  const int r = __ldg(idx + m);
-  if (!row_ok(r, N, flag)) return;
-  const float4* xl = reinterpret_cast<const float4*>(x_lat + static_cast<size_t>(r) * 16);
-  float xv[16];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const float4 a = __ldg(xl + q);
-    xv[4 * q] = a.x;
-    xv[4 * q + 1] = a.y;
-    xv[4 * q + 2] = a.z;
-    xv[4 * q + 3] = a.w;
-  }
-  float acc[4];
+// h[idx[m], j] = sum_c W_in[j, c] * x_lat[idx[m], c]; C = 16.  A thread owns
+// four hidden columns j0..j0+3: it loads their 64 weights once and reuses them
+// for kEmbedRows active rows, each row's 16 latent values being one broadcast
+// load for the whole warp; every row's four outputs are one 16-byte store
+// (a warp stores 512 contiguous bytes).
+constexpr int kEmbedRows = 16;
+constexpr int kEmbedThreads = 128;
+
+__global__ void __launch_bounds__(kEmbedThreads) k_embed(const float* __restrict__ w_in,
+                                                         const float* __restrict__ x_lat,
+                                                         const int32_t* __restrict__ idx, int n,
+                                                         int N, int D, float* __restrict__ h,
+                                                         int* flag) {
+  const int j0 = (blockIdx.x * kEmbedThreads + threadIdx.x) * 4;
+  if (j0 >= D) return;
+  float w[4][16];
 #pragma unroll
   for (int jj = 0; jj < 4; ++jj) {
     const float4* wr = reinterpret_cast<const float4*>(w_in + static_cast<size_t>(j0 + jj) * 16);
-    float s = 0.f;
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float4 w = __ldg(wr + q);
-      s = fmaf(w.x, xv[4 * q], s);
-      s = fmaf(w.y, xv[4 * q + 1], s);
-      s = fmaf(w.z, xv[4 * q + 2], s);
-      s = fmaf(w.w, xv[4 * q + 3], s);
+      const float4 v = __ldg(wr + q);
+      w[jj][4 * q] = v.x;
+      w[jj][4 * q + 1] = v.y;
+      w[jj][4 * q + 2] = v.z;
+      w[jj][4 * q + 3] = v.w;
     }
-    acc[jj] = s;
   }
-  *reinterpret_cast<float4*>(h + static_cast<size_t>(r) * D + j0) =
-      make_float4(acc[0], acc[1], acc[2], acc[3]);
+  const int m0 = blockIdx.y * kEmbedRows;
+  const int nm = min(n - m0, kEmbedRows);
+  int rows[kEmbedRows];  // all row indices first: independent loads
+#pragma unroll
+  for (int k = 0; k < kEmbedRows; ++k) rows[k] = k < nm ? __ldg(idx + m0 + k) : -1;
+#pragma unroll
+  for (int k = 0; k < kEmbedRows; ++k) {
+    const int r = rows[k];
+    if (k >= nm || !row_ok(r, N, flag)) continue;
+    const float4* xl = reinterpret_cast<const float4*>(x_lat + static_cast<size_t>(r) * 16);
+    float xv[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 a = __ldg(xl + q);
+      xv[4 * q] = a.x;
+      xv[4 * q + 1] = a.y;
+      xv[4 * q + 2] = a.z;
+      xv[4 * q + 3] = a.w;
+    }
+    float acc[4];
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      float s = 0.f;
+#pragma unroll
+      for (int c = 0; c < 16; ++c) s = fmaf(w[jj][c], xv[c], s);
+      acc[jj] = s;
+    }
+    *reinterpret_cast<float4*>(h + static_cast<size_t>(r) * D + j0) =
+        make_float4(acc[0], acc[1], acc[2], acc[3]);
+  }
 }
 
 cudaError_t launch_embed(const Ctx& c, const float* w_in, const float* x_lat, const int32_t* idx,
                          int n, float* h) {
   if (n <= 0) return cudaSuccess;
   Timed timed(c, TC_ROWS, static_cast<double>(n) * (64 + 4.0 * c.cfg.D));
-  const size_t total = static_cast<size_t>(n) * (c.cfg.D / 4);
-  k_embed<<<static_cast<unsigned>((total + 255) / 256), 256, 0, c.stream>>>(
-      w_in, x_lat, idx, n, c.cfg.N, c.cfg.D, h, c.flag);
+  const int D = c.cfg.D;
+  const dim3 grid((D / 4 + kEmbedThreads - 1) / kEmbedThreads, (n + kEmbedRows - 1) / kEmbedRows);
+  k_embed<<<grid, kEmbedThreads, 0, c.stream>>>(w_in, x_lat, idx, n, c.cfg.N, D, h, c.flag);
   c.launches += 1;
   return cudaGetLastError();
 }

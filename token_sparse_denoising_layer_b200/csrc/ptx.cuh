@@ -217,6 +217,23 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
       : "memory");
 }
 
+// The same load without the wait: the registers are valid only after
+// tmem_wait_ld(), so the next chunk can be in flight while this one is used.
+__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : HSA_R8(0), HSA_R8(8), HSA_R8(16), HSA_R8(24)
+      : "r"(taddr)
+      : "memory");
+}
+
+// Wait for every TMEM load this thread has issued.
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 #define HSA_R32(i) HSA_R8(i), HSA_R8(i + 8), HSA_R8(i + 16), HSA_R8(i + 24)
 
 // Load 64 consecutive fp32 columns of this thread's TMEM lane and wait.

@@ -143,10 +143,15 @@ class ShardRank:
         self.v_stage.zero_()
         abi.hsa_head(ctx, self.w_head, self.h, idx_r, nr, self.v_stage)
         yield ("all_reduce_sum", self.v_stage)
-        abi.hsa_euler_step(ctx, self.x, self.v_hat, self.v_hat_prev, self.v_stage, self.mask,
-                           float(self.sigmas[i]), float(self.sigmas[i + 1]))
+        s0, s1 = float(self.sigmas[i]), float(self.sigmas[i + 1])
         if regroup and self.T // self.budgets[-1] <= i < self.T - 1:
-            abi.hsa_select_groups(ctx, self.v_hat_prev, self.v_hat, self.score, self.g)
+            # the Euler pass also writes the re-grouping scores, as hsa_step does
+            abi.hsa_euler_step_score(ctx, self.x, self.v_hat, self.v_hat_prev, self.v_stage,
+                                     self.mask, s0, s1, self.score)
+            abi.hsa_select_from_score(ctx, self.score, self.g)
+        else:
+            abi.hsa_euler_step(ctx, self.x, self.v_hat, self.v_hat_prev, self.v_stage,
+                               self.mask, s0, s1)
 
     def n_active(self, i: int) -> int:
         return abi.hsa_n_active(self.ctx, i)
