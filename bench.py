@@ -1133,12 +1133,11 @@ def profile_case(name):
         for _ in range(3):
             abi.hsa_euler_step(ctx, x, vh, vp, vf, m, 0.5, 0.45)
     elif name == "rows":
-        # the HBM-bound row kernels, each on inputs larger than L2, two launches each:
-        # cached Euler over 4M tokens (1 GB of latent and velocities; the context's
-        # own scratch at the smallest width, D = 128, is 3.5 GB), the LN gather of
-        # all 32760 rows (D = 1536), and the KV scatter of 18900 rows into
-        # 75600 x 5120 caches
-        Ne = 4 * 1024 * 1024
+        # the HBM-bound row kernels on inputs larger than L2, two launches each:
+        # cached Euler over 1M tokens (256 MB of latent and velocities), the LN
+        # gather of all 32760 rows (D = 1536, 201 MB of fp32 rows), and the KV
+        # scatter of 16380 fresh rows into 32760 x 1536 caches
+        Ne = 1024 * 1024
         ce = abi.hsa_create(N=Ne, D=128, H=1, F=64, L=0, T=40, budgets=[40, 20, 10],
                             counts=[Ne - 2 * (Ne * 3 // 10), Ne * 3 // 10, Ne * 3 // 10])
         x, vh, vp, vf = (rnd(Ne, 16) for _ in range(4))
@@ -1154,15 +1153,12 @@ def profile_case(name):
         for _ in range(2):
             abi.hsa_ln_gather(ctx, h, idx, N, u)
         del h, u, idx
-        Nk, Dk, a = 75600, 5120, 18900
-        ck = abi.hsa_create(N=Nk, D=Dk, H=40, F=64, L=1, T=1, budgets=[1], counts=[Nk])
-        kr, vr = (rnd(a, Dk).to(torch.bfloat16) for _ in range(2))
-        kc, vc = (torch.zeros((Nk, Dk), dtype=torch.bfloat16, device="cuda") for _ in range(2))
-        ik = torch.sort(torch.randperm(Nk, generator=g, device="cuda")[:a]).values.to(torch.int32)
+        a = N // 2
+        kr, vr = (rnd(a, D).to(torch.bfloat16) for _ in range(2))
+        kc, vc = (torch.zeros((N, D), dtype=torch.bfloat16, device="cuda") for _ in range(2))
+        ik = torch.sort(torch.randperm(N, generator=g, device="cuda")[:a]).values.to(torch.int32)
         for _ in range(2):
-            abi.hsa_kv_scatter(ck, kr, vr, ik, a, kc, vc)
-        abi.hsa_sync_check(ck)
-        ck.close()
+            abi.hsa_kv_scatter(ctx, kr, vr, ik, a, kc, vc)
     elif name == "tokens":
         # the per-token kernels at the 21x45x80 latent (N = 75600, {40,20,10} at
         # 40/30/30%), two launches each: schedule (iteration 4: groups 1 and 2

@@ -274,3 +274,26 @@ def test_embed_and_head(N, D, a):
     assert normwise(vg[idx], O.head(w_head, hh[idx])) <= 1e-5
     assert (vg[rest] == 7.0).all()
     ctx.close()
+
+
+@pytest.mark.parametrize("direction", [1.0, -1.0])
+def test_attention_scores_that_grow_or_shrink_along_the_keys(direction):
+    """Scores that rise by about 32 log2 units per 128-key tile make the running
+    max fall behind again and again, so the kernel's rescale path (read S
+    again, raise the max, rescale O and l) runs repeatedly; falling scores put
+    the max in the first tile.  Both against the float64 oracle."""
+    need_gpu()
+    N, D, H, n = 1000, 128, 1, 200
+    ctx = _ctx(N, D, H, 64)
+    r = synth.rng(91)
+    q = synth.bf16_round(r.standard_normal((n, D), dtype=np.float32) * np.float32(0.1))
+    q[:, 0] = 8.0
+    K = synth.bf16_round(r.standard_normal((N, D), dtype=np.float32) * np.float32(0.1))
+    ramp = np.arange(N, dtype=np.float32) * np.float32(0.25)
+    K[:, 0] = synth.bf16_round(ramp if direction > 0 else ramp[::-1].copy())
+    V = synth.bf16_round(r.standard_normal((N, D), dtype=np.float32))
+    o = torch.empty((n, D), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_attention(ctx, bf(q), n, bf(K), bf(V), o)
+    abi.hsa_sync_check(ctx)
+    assert normwise(host(o), O.attention(q, K, V, H)) <= BF16_TOL
+    ctx.close()

@@ -14,9 +14,10 @@
 //   O_t += P_t V_j           tcgen05.mma with A = P_t read from TMEM
 // The two query tiles ping-pong: while warpgroup 0 turns S_0 into P_0, the
 // tensor core runs P_1 V and the next Q_1 K^T, and the other way round.
-// The running max m is raised only when a row's max grows by more than 2^8;
-// otherwise the stale max is kept, which is exact because the same m scales
-// both O and the row sum l.  A commit that signals S_t(j+1) also covers the
+// The running max m is set by the first key tile and raised only when a
+// tile's P would pass 2^64 (seen from its row sum, so no row-max pass precedes
+// the exponentials); otherwise the stale max is kept, which is exact because
+// the same m scales both O and the row sum l.  A commit that signals S_t(j+1) also covers the
 // earlier P_t(j) V_j, so softmax sees a stable O_t and a free P_t region.
 //
 // Warp 0: TMA producer.  Warp 1: TMEM owner and MMA issuer.  Warps 2..5 and
@@ -43,7 +44,6 @@ constexpr int kKV = 128;       // keys per tile
 constexpr int kStages = 2;     // K and V ring depth
 constexpr int kAttnThreads = 320;
 constexpr uint32_t kTmemCols = 512;
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
 
 template <int HD>
 struct AttnCfg {
@@ -75,6 +75,37 @@ struct AttnParams {
   float* part_o;     // [part][256 rows][HD] fp32, unnormalised
   float2* part_ml;   // [part][256 rows] (running max, row sum)
 };
+
+// Largest P (and so row sum) a tile may reach before the running max must be
+// raised: far inside the range of bf16 and of the fp32 row sums and O.
+constexpr float kSumLimit = 18446744073709551616.0f;  // 2^64
+
+__device__ __forceinline__ float row_max(const uint32_t (&sr)[kKV]) {
+  float mx[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) mx[u] = __uint_as_float(sr[u]);
+#pragma unroll
+  for (int e = 8; e < kKV; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sr[e]));
+  return fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+               fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+}
+
+// P = exp2(S*c - m) as bf16 pairs in w (packed f32x2 arithmetic: two lanes
+// per FMA/add instruction); returns the row sum of P.
+__device__ __forceinline__ float exp_row(const uint32_t (&sr)[kKV], float c, float m,
+                                         uint32_t (&w)[kKV / 2]) {
+  float rs0[4] = {0.f, 0.f, 0.f, 0.f}, rs1[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int e = 0; e < kKV; e += 2) {
+    float xa, xb;
+    fma2(xa, xb, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), c, -m);
+    const float a = ex2_approx(xa);
+    const float b = ex2_approx(xb);
+    add2(rs0[(e >> 1) & 3], rs1[(e >> 1) & 3], a, b);
+    w[e / 2] = pack_bf16(a, b);
+  }
+  return ((rs0[0] + rs1[0]) + (rs0[1] + rs1[1])) + ((rs0[2] + rs1[2]) + (rs0[3] + rs1[3]));
+}
 
 template <int HD>
 __global__ void __launch_bounds__(kAttnThreads, 1)
@@ -268,19 +299,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         for (int e = 0; e < kKV; ++e)
           if (e >= valid) sr[e] = __float_as_uint(-INFINITY);
       }
-      float mx[8];
+      // After the first tile the exponentials are taken against the running
+      // max as it stands, without a row-max pass first: any P below 2^64 is
+      // safe (bf16 and the fp32 sums hold it), and the row sum tells whether a
+      // value went past that.  Only then (rare) is S read again, its max taken,
+      // O and l rescaled and P recomputed.  The first tile takes the max first.
+      float m_use = m_run, alpha = 1.0f, rs;
+      if (j == 0) m_use = row_max(sr) * p.scale_log2;
+      uint32_t w[kKV / 2];
+#pragma unroll 1
+      for (int pass = 0;; ++pass) {
+        rs = exp_row(sr, p.scale_log2, m_use, w);
+        const bool over = !(rs <= kSumLimit);
+        if (j == 0 || pass == 1 || !__any_sync(0xffffffffu, over)) break;
+        // P is not stored yet, so S is still in TMEM: read it for its max,
+        // rescale O, then read it again for P (few live registers at a time)
+        tmem_ld128(tS, sr);
+        if (valid < kKV) {
 #pragma unroll
-      for (int u = 0; u < 8; ++u) mx[u] = __uint_as_float(sr[u]);
-#pragma unroll
-      for (int e = 8; e < kKV; ++e) mx[e & 7] = fmaxf(mx[e & 7], __uint_as_float(sr[e]));
-      float tmax = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-      tmax *= p.scale_log2;
-      const bool raise = tmax > m_run + kRescaleThreshold;
-      const float m_use = raise ? tmax : m_run;
-      const float alpha = raise ? ex2_approx(m_run - m_use) : 1.0f;
-      // O_t is stable here: the commit behind s_full covers P_t(j-1) V_{j-1}.
-      if (j > 0 && __any_sync(0xffffffffu, raise)) {
+          for (int e = 0; e < kKV; ++e)
+            if (e >= valid) sr[e] = __float_as_uint(-INFINITY);
+        }
+        const float tmax = row_max(sr) * p.scale_log2;
+        if (over) {
+          m_use = fmaxf(tmax, m_run);
+          alpha = ex2_approx(m_run - m_use);
+        }
+        // O_t is stable here: the commit behind s_full covers P_t(j-1) V_{j-1}.
 #pragma unroll 1
         for (int c = 0; c < HD / 32; ++c) {
           uint32_t r[32];
@@ -289,21 +334,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
           tmem_st32(tO + 32 * c, r);
         }
-      }
-      // P = exp2(S*c - m) as bf16 pairs, written over the S_t columns
-      // (packed f32x2 arithmetic: two lanes per FMA/add instruction)
-      uint32_t w[kKV / 2];
-      float rs0[4] = {0.f, 0.f, 0.f, 0.f}, rs1[4] = {0.f, 0.f, 0.f, 0.f};
+        tmem_ld128(tS, sr);
+        if (valid < kKV) {
 #pragma unroll
-      for (int e = 0; e < kKV; e += 2) {
-        float xa, xb;
-        fma2(xa, xb, __uint_as_float(sr[e]), __uint_as_float(sr[e + 1]), p.scale_log2, -m_use);
-        const float a = ex2_approx(xa);
-        const float b = ex2_approx(xb);
-        add2(rs0[(e >> 1) & 3], rs1[(e >> 1) & 3], a, b);
-        w[e / 2] = pack_bf16(a, b);
+          for (int e = 0; e < kKV; ++e)
+            if (e >= valid) sr[e] = __float_as_uint(-INFINITY);
+        }
       }
-      const float rs = ((rs0[0] + rs1[0]) + (rs0[1] + rs1[1])) + ((rs0[2] + rs1[2]) + (rs0[3] + rs1[3]));
       tmem_st64(tS, w);
       l_run = l_run * alpha + rs;
       m_run = m_use;

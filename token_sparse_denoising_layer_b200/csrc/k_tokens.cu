@@ -297,7 +297,8 @@ __global__ void __launch_bounds__(kSelThreads) k_radix_cut(const float* __restri
 // The same cut search with a cluster of kCutCluster CTAs per cut.  CTA c
 // holds the high words of the contiguous index range [c span, (c+1) span) in
 // shared memory; each radix pass sums the CTAs' 256-bin histograms through
-// distributed shared memory, so every CTA takes the same bin; the index
+// distributed shared memory, so every CTA takes the same bin (one cluster
+// barrier per pass: the histograms alternate between two buffers); the index
 // tie-break adds the CTAs' counts of keys equal to the final high word in
 // rank order.  Every CTA runs the same cluster barriers, and a last one keeps
 // each CTA's shared memory alive while the others read it.
@@ -322,7 +323,10 @@ __global__ void __cluster_dims__(kCutCluster, 1, 1) __launch_bounds__(kCutThread
     k_radix_cut_cluster(const float* __restrict__ score, int N, int span, CutParams cp,
                         uint32_t* cuts, int* flag) {
   extern __shared__ uint32_t skey[];  // [span]
-  __shared__ int hist[kRadixBins];    // this CTA's histogram, read by the cluster
+  // this CTA's histogram, read by the cluster; two buffers, alternating by
+  // pass, so a CTA may clear the next pass's buffer while others still read
+  // this pass's (they have all passed the barrier behind the one it clears)
+  __shared__ int hist2[2][kRadixBins];
   __shared__ int ghist[kRadixBins];   // the cluster's
   __shared__ int warp_sums[32];
   __shared__ uint32_t s_sel[2];
@@ -348,13 +352,15 @@ __global__ void __cluster_dims__(kCutCluster, 1, 1) __launch_bounds__(kCutThread
   int remaining = R;
   for (int pass = 0; pass < 4; ++pass) {
     const int shift = 24 - 8 * pass;
+    int* hist = hist2[pass & 1];
     for (int b = threadIdx.x; b < kRadixBins; b += blockDim.x) hist[b] = 0;
     __syncthreads();
     for (int i = threadIdx.x; i < cnt; i += blockDim.x) {
       const uint32_t h = skey[i];
       if ((h & pmask) == prefix) atomicAdd(&hist[(h >> shift) & 0xFF], 1);
     }
-    cluster_sync();  // every CTA's histogram is complete and visible
+    cluster_sync();  // every CTA's histogram is complete and visible, and every
+                     // CTA has finished reading the other buffer (two passes ago)
     for (int b = threadIdx.x; b < kRadixBins; b += blockDim.x) {
       const uint32_t a = smem_u32(&hist[b]);
       int sum = 0;
@@ -393,7 +399,6 @@ __global__ void __cluster_dims__(kCutCluster, 1, 1) __launch_bounds__(kCutThread
     remaining -= static_cast<int>(s_sel[1]);
     prefix |= bin << shift;
     pmask |= 0xFFu << shift;
-    cluster_sync();  // no CTA clears its histogram while another still reads it
   }
   // tie-break by index: the remaining-th key (0-based) whose high word is prefix
   int eq_local = 0;
