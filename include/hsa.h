@@ -277,6 +277,27 @@ hsa_status hsa_mlp_residual(hsa_ctx* ctx, const void* w_1, const void* w_2, floa
                             const int32_t* idx, int n);
 
 /*
+ * The stages above with the timestep modulation of a conditioned block (the
+ * reading of hsa_layer_forward_cond below; [TS] 2.2 step 4 names conditioning
+ * only as work skipped tokens do not incur), for callers that run a
+ * conditioned block stage by stage, such as a sequence-sharded step:
+ *   hsa_ln_gather_mod:            u[m] = LN(x[idx[m]]) * (1 + scale) + shift
+ *   hsa_out_proj_residual_gated:  x[idx[m]] += gate * (o[m] W_o^T)
+ *   hsa_mlp_residual_mod:         x[idx[m]] += gate * GELU(u2 W_1^T) W_2^T with
+ *                                 u2 = LN(x[idx[m]]) * (1 + scale) + shift
+ * shift, scale, gate (device) fp32 [D], 16-byte aligned; shift and scale are
+ * both given or both NULL (no modulation), gate NULL means 1.  Other
+ * arguments, layouts and errors as the unmodulated calls.
+ */
+hsa_status hsa_ln_gather_mod(hsa_ctx* ctx, const float* x, const int32_t* idx, int n, void* u,
+                             const float* shift, const float* scale);
+hsa_status hsa_out_proj_residual_gated(hsa_ctx* ctx, const void* w_o, const void* o,
+                                       const int32_t* idx, int n, float* x, const float* gate);
+hsa_status hsa_mlp_residual_mod(hsa_ctx* ctx, const void* w_1, const void* w_2, float* x,
+                                const int32_t* idx, int n, const float* shift,
+                                const float* scale, const float* gate);
+
+/*
  * One transformer block on the active set ([TS] 2.2): LN -> QKV (K/V written
  * into the caches) -> attention of the n queries against all N cached rows
  * -> out-projection + residual -> LN -> MLP + residual.  Only rows idx of x

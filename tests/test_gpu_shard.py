@@ -151,3 +151,54 @@ def test_sharded_world_of_one_through_nccl():
         rk.close()
     finally:
         dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("G", [1, 2, 3])
+def test_sharded_conditioned_step(G):
+    """Conditioned blocks (per-iteration modulation of every layer, text
+    cross-attention in every layer) in the sharded step: every rank ends with
+    the same latent bit for bit, equal to the single-GPU conditioned loop
+    (hsa_step_cond) within rounding, and to the float64 oracle within 2e-2."""
+    need_gpu()
+    from token_sparse_denoising_layer_b200.loop import HsaLoop
+    from token_sparse_denoising_layer_b200.shard import ShardRank, run_local
+
+    spec, sh, counts, w, layers = _model("tiny_dit")
+    T, L = spec["T"], sh.L
+    mods = [[synth.modulation(sh.D, 300 + i * L + l, spread=0.3) for l in range(L)]
+            for i in range(T)]
+    cross = [synth.cross_attention_weights(sh.D, 16, 400 + l) for l in range(L)]
+    mods_dev = [[dev(m) for m in row] for row in mods]
+    xa = [abi.cross_attn(bf(c["w_q"]), bf(c["w_o"]), bf(c["k_txt"]), bf(c["v_txt"]), 16)
+          for c in cross]
+    conds = [abi.StepCond(mods_dev[i], xa) for i in range(T)]
+    x0 = synth.latent(sh.N, 16, 9)
+    g0 = synth.random_split(sh.N, counts, 9)
+    ranks = [ShardRank(r, G, sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]),
+                       T, spec["budgets"], counts, shift=spec["shift"]) for r in range(G)]
+    for rk in ranks:
+        rk.reset(dev(x0), dev(g0))
+    for i in range(T):
+        run_local([rk.steps(i, True, cond=conds[i]) for rk in ranks])
+    for rk in ranks:
+        abi.hsa_sync_check(rk.ctx)
+    xs = [host(rk.x) for rk in ranks]
+    for rk in ranks:
+        rk.close()
+    for r in range(1, G):
+        assert np.array_equal(xs[r], xs[0])
+    loop = HsaLoop(sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]), T,
+                   spec["budgets"], counts, shift=spec["shift"])
+    loop.reset(x0, g0)
+    for i in range(T):
+        loop.step(i, True, cond=conds[i])
+    abi.hsa_sync_check(loop.ctx)
+    x1 = host(loop.x)
+    loop.close()
+    d = _rel(xs[0], x1)
+    print(f"conditioned, G={G}: sharded vs single-GPU loop {d:.2e} "
+          f"(bitwise: {np.array_equal(xs[0], x1)})")
+    assert d <= 1e-2
+    xr = O.run_loop(w, x0, g0, T, list(spec["budgets"]), counts,
+                    O.sigma_schedule(T, spec["shift"]), sh.H, mods=mods, cross=cross)
+    assert _rel(xs[0], xr) <= 2e-2

@@ -21,6 +21,7 @@ SYMBOLS = [
     "hsa_selftest_timeout", "hsa_kernel_launches", "hsa_time_kernels", "hsa_kernel_times", "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
     "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_linear", "hsa_kv_scatter", "hsa_kv_scatter_packed",
     "hsa_attention", "hsa_attention_kv", "hsa_out_proj_residual", "hsa_mlp_residual",
+    "hsa_ln_gather_mod", "hsa_out_proj_residual_gated", "hsa_mlp_residual_mod",
     "hsa_layer_forward", "hsa_layer_forward_cond", "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_euler_step_score", "hsa_step", "hsa_step_cond",
     "hsa_select_groups_static",
 ]
@@ -116,6 +117,9 @@ def load() -> ctypes.CDLL:
         "hsa_attention_kv": (I, [P, P, I, P, P, I, P]),
         "hsa_out_proj_residual": (I, [P, P, P, P, I, P]),
         "hsa_mlp_residual": (I, [P, P, P, P, P, I]),
+        "hsa_ln_gather_mod": (I, [P, P, P, I, P, P, P]),
+        "hsa_out_proj_residual_gated": (I, [P, P, P, P, I, P, P]),
+        "hsa_mlp_residual_mod": (I, [P, P, P, P, P, I, P, P, P]),
         "hsa_layer_forward": (I, [P, ctypes.POINTER(hsa_layer_weights), P, P, I, P, P]),
         "hsa_layer_forward_cond": (I, [P, ctypes.POINTER(hsa_layer_weights), P,
                                        ctypes.POINTER(hsa_cross_attn), P, P, I, P, P]),
@@ -286,6 +290,26 @@ def hsa_out_proj_residual(ctx: Context, w_o, o, idx, n: int, x) -> None:
 
 def hsa_mlp_residual(ctx: Context, w_1, w_2, x, idx, n: int) -> None:
     _check(ctx.ptr, load().hsa_mlp_residual(ctx.ptr, _p(w_1), _p(w_2), _p(x), _p(idx), n))
+
+
+def _opt(t):
+    return _p(t) if t is not None else None
+
+
+def hsa_ln_gather_mod(ctx: Context, x, idx, n: int, u, shift=None, scale=None) -> None:
+    _check(ctx.ptr, load().hsa_ln_gather_mod(ctx.ptr, _p(x), _p(idx), n, _p(u), _opt(shift),
+                                             _opt(scale)))
+
+
+def hsa_out_proj_residual_gated(ctx: Context, w_o, o, idx, n: int, x, gate=None) -> None:
+    _check(ctx.ptr, load().hsa_out_proj_residual_gated(ctx.ptr, _p(w_o), _p(o), _p(idx), n,
+                                                       _p(x), _opt(gate)))
+
+
+def hsa_mlp_residual_mod(ctx: Context, w_1, w_2, x, idx, n: int, shift=None, scale=None,
+                         gate=None) -> None:
+    _check(ctx.ptr, load().hsa_mlp_residual_mod(ctx.ptr, _p(w_1), _p(w_2), _p(x), _p(idx), n,
+                                                _opt(shift), _opt(scale), _opt(gate)))
 
 
 def layer_weights(w_qkv, w_o, w_1, w_2) -> hsa_layer_weights:

@@ -503,6 +503,55 @@ hsa_status hsa_out_proj_residual(hsa_ctx* ctx, const void* w_o, const void* o,
 }
 
 
+hsa_status hsa_out_proj_residual_gated(hsa_ctx* ctx, const void* w_o, const void* o,
+                                       const int32_t* idx, int n, float* x, const float* gate) {
+  HSA_CHECK_CTX(ctx);
+  if (hsa_status st = check_n(ctx, n)) return st;
+  if (gate != nullptr && (reinterpret_cast<uintptr_t>(gate) & 15) != 0)
+    return fail(ctx, HSA_ERR_INVALID_ARG, "gate must be 16-byte aligned");
+  if (n == 0) return HSA_OK;
+  HSA_CHECK_PTR(ctx, w_o);
+  HSA_CHECK_PTR(ctx, o);
+  HSA_CHECK_PTR(ctx, idx);
+  HSA_CHECK_PTR(ctx, x);
+  return proj_residual(ctx, w_o, o, idx, n, x, gate, "out_proj");
+}
+
+hsa_status hsa_ln_gather_mod(hsa_ctx* ctx, const float* x, const int32_t* idx, int n, void* u,
+                             const float* shift, const float* scale) {
+  HSA_CHECK_CTX(ctx);
+  if (hsa_status st = check_n(ctx, n)) return st;
+  if ((shift == nullptr) != (scale == nullptr))
+    return fail(ctx, HSA_ERR_INVALID_ARG, "shift and scale are given together or not at all");
+  if (shift != nullptr) {
+    HSA_CHECK_PTR(ctx, shift);
+    HSA_CHECK_PTR(ctx, scale);
+  }
+  if (n == 0) return HSA_OK;
+  HSA_CHECK_PTR(ctx, x);
+  HSA_CHECK_PTR(ctx, idx);
+  HSA_CHECK_PTR(ctx, u);
+  return launched(ctx, hsa::launch_ln_gather(ctx->c, x, idx, n, u, shift, scale), "ln_gather");
+}
+
+hsa_status hsa_mlp_residual_mod(hsa_ctx* ctx, const void* w_1, const void* w_2, float* x,
+                                const int32_t* idx, int n, const float* shift,
+                                const float* scale, const float* gate) {
+  HSA_CHECK_CTX(ctx);
+  if (hsa_status st = check_n(ctx, n)) return st;
+  if ((shift == nullptr) != (scale == nullptr))
+    return fail(ctx, HSA_ERR_INVALID_ARG, "shift and scale are given together or not at all");
+  for (const float* v : {shift, scale, gate})
+    if (v != nullptr && (reinterpret_cast<uintptr_t>(v) & 15) != 0)
+      return fail(ctx, HSA_ERR_INVALID_ARG, "modulation rows must be 16-byte aligned");
+  if (n == 0) return HSA_OK;
+  HSA_CHECK_PTR(ctx, w_1);
+  HSA_CHECK_PTR(ctx, w_2);
+  HSA_CHECK_PTR(ctx, x);
+  HSA_CHECK_PTR(ctx, idx);
+  return mlp_residual(ctx, w_1, w_2, x, idx, n, shift, scale, gate);
+}
+
 hsa_status hsa_mlp_residual(hsa_ctx* ctx, const void* w_1, const void* w_2, float* x,
                             const int32_t* idx, int n) {
   HSA_CHECK_CTX(ctx);

@@ -19,7 +19,8 @@ the cache by A_i.
 Per step on rank r:
   schedule (all of A_i) -> embed, L x [LN, Q and K|V GEMMs of its chunk,
   all-gather K|V, scatter into the cache, attention of its queries against
-  all N rows, out-projection + MLP] -> head of its chunk into a zeroed [N, C]
+  all N rows, out-projection, (text cross-attention), MLP; with the
+  iteration's modulation when conditioned] -> head of its chunk into a zeroed [N, C]
   buffer -> all-reduce (sum) of that buffer, which is exact because every
   active row has exactly one non-zero contributor -> cached Euler over all N
   (replicated) -> re-grouping (replicated; deterministic, so the group ids
@@ -121,9 +122,16 @@ class ShardRank:
         for buf in (self.v_hat, self.v_hat_prev, self.v_stage, self.score):
             buf.zero_()
 
-    def steps(self, i: int, regroup: bool = True) -> Iterator[Request]:
-        """Global iteration i on this rank; yields at each exchange."""
+    def steps(self, i: int, regroup: bool = True, cond=None) -> Iterator[Request]:
+        """Global iteration i on this rank; yields at each exchange.
+
+        ``cond`` (abi.StepCond, or None) conditions the blocks as hsa_step_cond
+        does: layer l's modulation rows of this iteration and its text
+        cross-attention, run on the rank's own active rows (the text keys and
+        values are the same on every rank, so cross-attention needs no
+        exchange)."""
         ctx, D = self.ctx, self.D
+        mods, cross = cond._keep if cond is not None else (None, None)
         a = abi.hsa_schedule(ctx, i, self.g, self.mask, self.active_idx)
         c, sl = shard_slices(a, self.G)
         s0, nr = sl[self.rank]
@@ -131,15 +139,24 @@ class ShardRank:
         abi.hsa_embed(ctx, self.w_in, self.x, idx_r, nr, self.h)
         for l in range(self.L):
             _, w_o, w_1, w_2 = self.layers[l]
-            abi.hsa_ln_gather(ctx, self.h, idx_r, nr, self.u)
+            m = None if mods is None else mods[l]   # rows shift_a, scale_a, gate_a, shift_m, ...
+            row = (lambda r: None) if m is None else (lambda r, m=m: m[r])
+            abi.hsa_ln_gather_mod(ctx, self.h, idx_r, nr, self.u, row(0), row(1))
             abi.hsa_linear(ctx, self.u, nr, D, self.w_q[l], D, self.q)
             abi.hsa_linear(ctx, self.u, nr, D, self.w_kv[l], 2 * D, self.kv_send)
             yield ("all_gather", self.kv_send[:c], self.kv_recv[:self.G * c])
             abi.hsa_kv_scatter_packed(ctx, self.kv_recv, self.active_idx, a, self.k_cache[l],
                                       self.v_cache[l])
             abi.hsa_attention(ctx, self.q, nr, self.k_cache[l], self.v_cache[l], self.o)
-            abi.hsa_out_proj_residual(ctx, w_o, self.o, idx_r, nr, self.h)
-            abi.hsa_mlp_residual(ctx, w_1, w_2, self.h, idx_r, nr)
+            abi.hsa_out_proj_residual_gated(ctx, w_o, self.o, idx_r, nr, self.h, row(2))
+            xa = None if cross is None else cross[l]
+            if xa is not None:
+                w_qc, w_oc, k_txt, v_txt = xa._keep
+                abi.hsa_ln_gather(ctx, self.h, idx_r, nr, self.u)
+                abi.hsa_linear(ctx, self.u, nr, D, w_qc, D, self.q)
+                abi.hsa_attention_kv(ctx, self.q, nr, k_txt, v_txt, xa.n_txt, self.o)
+                abi.hsa_out_proj_residual(ctx, w_oc, self.o, idx_r, nr, self.h)
+            abi.hsa_mlp_residual_mod(ctx, w_1, w_2, self.h, idx_r, nr, row(3), row(4), row(5))
         self.v_stage.zero_()
         abi.hsa_head(ctx, self.w_head, self.h, idx_r, nr, self.v_stage)
         yield ("all_reduce_sum", self.v_stage)
