@@ -217,14 +217,10 @@ __global__ void __launch_bounds__(kEmbedThreads) k_embed(const float* __restrict
     }
   }
   const int m0 = blockIdx.y * kEmbedRows;
-  const int nm = min(n - m0, kEmbedRows);
-  int rows[kEmbedRows];  // all row indices first: independent loads
-#pragma unroll
-  for (int k = 0; k < kEmbedRows; ++k) rows[k] = k < nm ? __ldg(idx + m0 + k) : -1;
-#pragma unroll
-  for (int k = 0; k < kEmbedRows; ++k) {
-    const int r = rows[k];
-    if (k >= nm || !row_ok(r, N, flag)) continue;
+  const int m1 = min(n, m0 + kEmbedRows);
+  for (int m = m0; m < m1; ++m) {
+    const int r = __ldg(idx + m);
+    if (!row_ok(r, N, flag)) continue;
     const float4* xl = reinterpret_cast<const float4*>(x_lat + static_cast<size_t>(r) * 16);
     float xv[16];
 #pragma unroll
