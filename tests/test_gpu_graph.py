@@ -54,3 +54,32 @@ def test_replay_needs_capture():
     with pytest.raises(RuntimeError):
         loop.replay()
     loop.close()
+
+
+def test_kernel_times_count_and_work_per_class():
+    """hsa_time_kernels: one step of the tiny DiT with every launch timed. Per
+    class the call counts follow the step's structure and the attention and
+    GEMM work is the algorithmic FLOP of the step (4 a N D per attention, 2 M
+    Ncols K per GEMM); reading clears the totals."""
+    need_gpu()
+    loop, x0, g0 = _loop("tiny_dit")
+    loop.reset(x0, g0)
+    abi.hsa_kernel_times(loop.ctx)
+    abi.hsa_time_kernels(loop.ctx, True)
+    loop.step(0)
+    kt = abi.hsa_kernel_times(loop.ctx)
+    abi.hsa_time_kernels(loop.ctx, False)
+    abi.hsa_sync_check(loop.ctx)
+    N, D, F, L = loop.N, loop.D, loop.F, loop.L
+    a = loop.n_active(0)
+    assert kt["attention"]["calls"] == L
+    assert kt["gemm"]["calls"] == 4 * L
+    assert kt["rows"]["calls"] == 2 * L + 2          # LN gathers, embed, head
+    assert kt["tokens"]["calls"] == 2                # schedule, Euler
+    assert kt["attention"]["work"] == L * 4.0 * a * N * D
+    assert kt["gemm"]["work"] == L * 2.0 * a * (3 * D * D + D * D + 2 * D * F)
+    for v in kt.values():
+        assert v["ms"] > 0
+    again = abi.hsa_kernel_times(loop.ctx)
+    assert all(v["calls"] == 0 and v["ms"] == 0 for v in again.values())
+    loop.close()
