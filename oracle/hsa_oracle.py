@@ -16,8 +16,10 @@ Each function cites the passage it follows.  Sources:
 Where the pages are silent, the plainest reading is taken and named in the
 docstring ("reading: ...").  Parity status per function:
   pinned   - checked in tests against closed forms, brute force or invariants
-  unpinned - ``sigma_schedule`` beyond its endpoints, the shift form, and the
-             re-grouping cadence in ``run_loop`` (a chosen convention).
+  readings - the shift form of ``sigma_schedule`` and the re-grouping cadence
+             in ``run_loop`` are conventions the pages leave open; the code
+             is pinned to them (the shift by its odds identity, the cadence
+             by its first re-grouping step).
 """
 
 from __future__ import annotations
@@ -161,7 +163,7 @@ def assign_groups(score: np.ndarray, counts: Sequence[int]) -> np.ndarray:
 # --------------------------------------------------------------------------
 
 def sigma_schedule(T: int, shift: float = 1.0) -> np.ndarray:
-    """Noise levels sigma_0..sigma_T as float32 (parity unpinned beyond endpoints).
+    """Noise levels sigma_0..sigma_T as float32.
 
     Reading: linear sigma_j = 1 - j/T, then the flow-matching timestep shift
     sigma' = s*sigma / (1 + (s-1)*sigma); computed in float64, rounded to float32.

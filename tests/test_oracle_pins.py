@@ -492,6 +492,21 @@ def test_euler_f32_matches_f64_within_rounding():
     assert (a[1] == b[1]).all() and (a[2] == b[2]).all()
 
 
+def test_sigma_shift_scales_the_odds():
+    """The flow-matching timestep shift by a factor s multiplies the odds of
+    every interior noise level by s: sigma' / (1 - sigma') = s sigma / (1 - sigma)
+    with sigma = 1 - j/T (exact rationals; the table is float32).  A shift by
+    1/s instead of s, or a shift of 1 - sigma, breaks it."""
+    T = 40
+    for shift in (5.0, 3.0):
+        tab = O.sigma_schedule(T, shift)
+        for j in range(1, T):
+            sig = Fraction(T - j, T)
+            odds = Fraction(int(shift)) * sig / (1 - sig)
+            want = odds / (1 + odds)
+            assert abs(Fraction(float(tab[j])) - want) <= Fraction(1, 2 ** 23), (shift, j)
+
+
 def test_sigma_schedule_endpoints_and_monotone():
     for shift in (1.0, 5.0):
         s = O.sigma_schedule(40, shift)
