@@ -933,10 +933,19 @@ def run_ours(args, rank, world, local, pg):
                     "ms_per_launch": round(at["ms"] / max(at["calls"], 1), 4),
                     "per_launch": "4*|A_i|*N*D FLOP, N = 32760, D = 1536; |A_i| = 32760, "
                                   "22932 or 13104 by iteration (6.594 TFLOP at |A_i| = N)",
-                    "traffic": attention_traffic(),
-                    "traffic_case": "ncu capture of one launch at |A| = N = 32760",
-                    "algorithmic_bytes": 4 * 32760 * 1536 * 2,
                     "burst_peak": peak_burst}
+            # bytes of the average attention launch of the step: Q and O rows
+            # (2 B x D each per active row) and the K, V cache (2 B x D each per row)
+            a_avg = at["work"] / (4.0 * sh.N * sh.D) / max(at["calls"], 1)
+            algo_avg = 4.0 * sh.D * (a_avg + sh.N)
+            algo_full = 4.0 * sh.D * (sh.N + sh.N)
+            t_full = attention_traffic()
+            roof["algorithmic_bytes"] = round(algo_avg)
+            roof["traffic"] = round(t_full * algo_avg / algo_full) if t_full is not None else None
+            roof["traffic_note"] = ("ncu DRAM bytes (read + write) of one launch at |A| = N = 32760 "
+                                    f"({t_full} B against {round(algo_full)} B algorithmic), "
+                                    "scaled to the step's average launch by its algorithmic bytes"
+                                    if t_full is not None else "no capture of the current kernel")
             if "attention" in sub:
                 a100 = sub["attention"]["100%"]
                 roof["isolated_100pct"] = {"tflops": a100["tflops"],

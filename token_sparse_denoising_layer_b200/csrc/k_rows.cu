@@ -256,56 +256,84 @@ cudaError_t launch_embed(const Ctx& c, const float* w_in, const float* x_lat, co
 }
 
 // ------------------------------------------------------------ velocity head
-// One warp per active row: v_fresh[idx[m], o] = sum_j LN(h[idx[m]])_j W_head[o, j].
-// fp32 throughout; the 16 dot products are reduced with butterflies.
-__global__ void __launch_bounds__(256) k_head(const float* __restrict__ w_head,
+// v_fresh[idx[m], o] = sum_j LN(h[idx[m]])_j W_head[o, j], fp32 throughout.
+// One warp takes kHeadRows active rows: the statistics of each row come from
+// two passes over it (mean, then the centred sum of squares), and the dot
+// products with the 16 rows of W_head read each W_head vector once for all of
+// the warp's rows, so W_head's L1 traffic is shared kHeadRows ways.  The 16
+// sums of each row are reduced with butterflies.
+constexpr int kHeadRows = 4;
+
+__global__ void __launch_bounds__(128) k_head(const float* __restrict__ w_head,
                                               const float* __restrict__ h,
                                               const int32_t* __restrict__ idx, int n, int N,
                                               int D, float* __restrict__ v_fresh, int* flag) {
-  const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int m0 = (blockIdx.x * 4 + (threadIdx.x >> 5)) * kHeadRows;
   const int lane = threadIdx.x & 31;
-  if (m >= n) return;
-  const int r = __ldg(idx + m);
-  if (!row_ok(r, N, flag)) return;
-  const float4* hr = reinterpret_cast<const float4*>(h + static_cast<size_t>(r) * D);
+  if (m0 >= n) return;
   const int nv = D / 4;
-  float s = 0.f;
-  for (int c = lane; c < nv; c += 32) {
-    const float4 a = __ldg(hr + c);
-    s += (a.x + a.y) + (a.z + a.w);
-  }
-  const float mean = warp_sum(s) / static_cast<float>(D);
-  float q = 0.f;
-  for (int c = lane; c < nv; c += 32) {
-    const float4 a = __ldg(hr + c);
-    const float p0 = a.x - mean, p1 = a.y - mean, p2 = a.z - mean, p3 = a.w - mean;
-    q += (p0 * p0 + p1 * p1) + (p2 * p2 + p3 * p3);
-  }
-  const float rstd = 1.0f / sqrtf(warp_sum(q) / static_cast<float>(D) + kLnEps);
-  float acc[16];
+  const float4* hr[kHeadRows];
+  int r[kHeadRows];
+  bool use[kHeadRows];
 #pragma unroll
-  for (int o = 0; o < 16; ++o) acc[o] = 0.f;
+  for (int k = 0; k < kHeadRows; ++k) {
+    r[k] = m0 + k < n ? __ldg(idx + m0 + k) : 0;
+    use[k] = m0 + k < n && row_ok(r[k], N, flag);
+    hr[k] = reinterpret_cast<const float4*>(h + static_cast<size_t>(use[k] ? r[k] : 0) * D);
+  }
+  float mean[kHeadRows], rstd[kHeadRows];
+#pragma unroll
+  for (int k = 0; k < kHeadRows; ++k) {
+    float s = 0.f;
+    for (int c = lane; c < nv; c += 32) {
+      const float4 a = __ldg(hr[k] + c);
+      s += (a.x + a.y) + (a.z + a.w);
+    }
+    mean[k] = warp_sum(s) / static_cast<float>(D);
+    float q = 0.f;
+    for (int c = lane; c < nv; c += 32) {
+      const float4 a = __ldg(hr[k] + c);
+      const float p0 = a.x - mean[k], p1 = a.y - mean[k], p2 = a.z - mean[k], p3 = a.w - mean[k];
+      q += (p0 * p0 + p1 * p1) + (p2 * p2 + p3 * p3);
+    }
+    rstd[k] = 1.0f / sqrtf(warp_sum(q) / static_cast<float>(D) + kLnEps);
+  }
+  float acc[kHeadRows][16];
+#pragma unroll
+  for (int k = 0; k < kHeadRows; ++k)
+#pragma unroll
+    for (int o = 0; o < 16; ++o) acc[k][o] = 0.f;
   for (int c = lane; c < nv; c += 32) {
-    float4 a = __ldg(hr + c);
-    a.x = (a.x - mean) * rstd;
-    a.y = (a.y - mean) * rstd;
-    a.z = (a.z - mean) * rstd;
-    a.w = (a.w - mean) * rstd;
+    float4 a[kHeadRows];
+#pragma unroll
+    for (int k = 0; k < kHeadRows; ++k) {
+      a[k] = __ldg(hr[k] + c);
+      a[k].x = (a[k].x - mean[k]) * rstd[k];
+      a[k].y = (a[k].y - mean[k]) * rstd[k];
+      a[k].z = (a[k].z - mean[k]) * rstd[k];
+      a[k].w = (a[k].w - mean[k]) * rstd[k];
+    }
 #pragma unroll
     for (int o = 0; o < 16; ++o) {
       const float4 w = __ldg(reinterpret_cast<const float4*>(w_head + static_cast<size_t>(o) * D) + c);
-      acc[o] = fmaf(a.x, w.x, fmaf(a.y, w.y, fmaf(a.z, w.z, fmaf(a.w, w.w, acc[o]))));
+#pragma unroll
+      for (int k = 0; k < kHeadRows; ++k)
+        acc[k][o] = fmaf(a[k].x, w.x, fmaf(a[k].y, w.y, fmaf(a[k].z, w.z, fmaf(a[k].w, w.w, acc[k][o]))));
     }
   }
 #pragma unroll
-  for (int o = 0; o < 16; ++o) acc[o] = warp_sum(acc[o]);
-  if (lane < 4) {
-    // lane l writes channels 4l..4l+3 (constant register indices)
-    float4 outv = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int k = 0; k < kHeadRows; ++k) {
 #pragma unroll
-    for (int l = 0; l < 4; ++l)
-      if (lane == l) outv = make_float4(acc[4 * l], acc[4 * l + 1], acc[4 * l + 2], acc[4 * l + 3]);
-    reinterpret_cast<float4*>(v_fresh + static_cast<size_t>(r) * 16)[lane] = outv;
+    for (int o = 0; o < 16; ++o) acc[k][o] = warp_sum(acc[k][o]);
+    if (use[k] && lane < 4) {
+      // lane l writes channels 4l..4l+3 (constant register indices)
+      float4 outv = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+      for (int l = 0; l < 4; ++l)
+        if (lane == l)
+          outv = make_float4(acc[k][4 * l], acc[k][4 * l + 1], acc[k][4 * l + 2], acc[k][4 * l + 3]);
+      reinterpret_cast<float4*>(v_fresh + static_cast<size_t>(r[k]) * 16)[lane] = outv;
+    }
   }
 }
 
@@ -313,7 +341,9 @@ cudaError_t launch_head(const Ctx& c, const float* w_head, const float* h, const
                         int n, float* v_fresh) {
   if (n <= 0) return cudaSuccess;
   Timed timed(c, TC_ROWS, static_cast<double>(n) * (4.0 * c.cfg.D + 64));
-  k_head<<<(n + 7) / 8, 256, 0, c.stream>>>(w_head, h, idx, n, c.cfg.N, c.cfg.D, v_fresh, c.flag);
+  const int warps = (n + kHeadRows - 1) / kHeadRows;
+  k_head<<<(warps + 3) / 4, 128, 0, c.stream>>>(w_head, h, idx, n, c.cfg.N, c.cfg.D, v_fresh,
+                                                 c.flag);
   c.launches += 1;
   return cudaGetLastError();
 }
