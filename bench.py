@@ -50,6 +50,9 @@ def parse():
                     help="replicas: one loop per GPU (weak scaling); shard: one loop split "
                          "over the GPUs by active-list chunks with a K/V all-gather per layer "
                          "(strong scaling)")
+    ap.add_argument("--kv-exchange", choices=["gather", "peer"], default="gather",
+                    help="shard mode: K|V rows by NCCL all-gather + scatter, or stored by the "
+                         "QKV GEMM's epilogue straight into every rank's cache (peer memory)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the sub-benchmarks (profiling runs)")
     ap.add_argument("--profile-case", choices=["attention", "gemm", "euler", "rows", "tokens",
@@ -990,7 +993,8 @@ def run_shard(args, rank, world, local, pg):
     import torch
 
     from token_sparse_denoising_layer_b200 import abi, synth
-    from token_sparse_denoising_layer_b200.shard import ShardRank, run_dist, run_local
+    from token_sparse_denoising_layer_b200.shard import (ShardRank, link_local, link_symmetric,
+                                                         run_dist, run_local)
 
     torch.cuda.set_device(local)
     spec = synth.WORKLOADS[WORKLOAD]
@@ -1002,6 +1006,11 @@ def run_shard(args, rank, world, local, pg):
     rk = ShardRank(rank, world, sh.N, sh.D, sh.H, sh.F, layers,
                    torch.from_numpy(wf["w_in"]).cuda(), torch.from_numpy(wf["w_head"]).cuda(),
                    spec["T"], spec["budgets"], counts, shift=spec["shift"])
+    if args.kv_exchange == "peer":
+        if pg is not None:
+            link_symmetric(rk, pg)
+        else:
+            link_local([rk])
     x0 = torch.from_numpy(synth.latent(sh.N, 16, 0)).cuda()
     g0 = torch.from_numpy(synth.random_split(sh.N, counts, 0)).cuda()
 
@@ -1057,8 +1066,10 @@ def run_shard(args, rank, world, local, pg):
             "data": "synthetic (seeded; random N(0,1/fan_in) weights, x ~ N(0,1))",
             "config": {"workload": ORACLE_WORKLOAD,
                        "global_batch": 1, "seq_len": sh.N,
-                       "parallelism": f"sequence-shard x{world} (active-list chunks, K|V "
-                                      f"all-gather per layer, velocity all-reduce per step)",
+                       "parallelism": f"sequence-shard x{world} (active-list chunks, " + (
+                           "K|V all-gather per layer" if args.kv_exchange == "gather" else
+                           "K|V stored into every rank's cache by the QKV epilogue + barrier "
+                           "per layer") + ", velocity all-reduce per step)",
                        "l2": "inputs larger than L2 (>8 GB touched per step)",
                        "step": "one global iteration i = k mod 40; 40 steps = one loop",
                        "value": "ms per step of the one loop, max over ranks"},

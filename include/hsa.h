@@ -212,6 +212,30 @@ hsa_status hsa_qkv_project(hsa_ctx* ctx, const void* w_qkv, const void* u, const
                            int n, void* q, void* k_cache, void* v_cache);
 
 /*
+ * The same QKV projection for a sequence-sharded step, with the exchange of
+ * the fresh K/V rows folded into the GEMM's epilogue ([TS] 2.2 steps 1-2:
+ * every active token's fresh K/V rows must reach every copy of the cache
+ * before attention reads it).  Q goes to q as in hsa_qkv_project; every fresh
+ * K and V row is stored to row idx[m] of each of the n_caches cache pairs,
+ * so that one launch writes this rank's rows into its own cache and, through
+ * peer-mapped pointers, into every other rank's copy over NVLink.
+ *   w_qkv, u, idx, q as hsa_qkv_project;
+ *   k_caches, v_caches (HOST arrays of n_caches pointers, borrowed for the
+ *   call): device bf16 [N, D] caches, each on this GPU or a peer GPU's memory
+ *   mapped into this process (P2P or symmetric memory); 1 <= n_caches <= 8.
+ * The launch only stores to peer memory (no load reads another GPU).  The
+ * caller orders it against the peers' readers: no peer may read the rows
+ * before this launch completes (a device-side barrier on the stream after
+ * it), and no peer may still be reading a previous step's rows of these
+ * caches when it starts.  HSA_ERR_INVALID_ARG for n_caches out of range or a
+ * NULL / misaligned pointer; an index outside [0, N) is skipped and reported
+ * by hsa_sync_check (HSA_ERR_DEVICE_CHECK).
+ */
+hsa_status hsa_qkv_project_peers(hsa_ctx* ctx, const void* w_qkv, const void* u,
+                                 const int32_t* idx, int n, void* q, void* const* k_caches,
+                                 void* const* v_caches, int n_caches);
+
+/*
  * Active-row linear map, the tensor-core building block of the QKV,
  * out-projection and MLP products ([TS] 2.2): out = a w^T, fp32 accumulation.
  *   a (device) bf16 [M, Kd];  w (device) bf16 [Ncols, Kd];  out (device) bf16 [M, Ncols].

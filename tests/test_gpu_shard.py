@@ -14,7 +14,7 @@ import socket
 import numpy as np
 import pytest
 
-from gpu_util import bf, dev, host, need_gpu, torch
+from gpu_util import BF16_TOL, bf, dev, host, need_gpu, normwise, torch
 from oracle import hsa_oracle as O
 from token_sparse_denoising_layer_b200 import abi, synth
 
@@ -49,11 +49,13 @@ def _model(name, N=None, L=None):
     return spec, sh, counts, w, layers
 
 
-def _run_sharded(G, spec, sh, counts, w, layers, regroup):
-    from token_sparse_denoising_layer_b200.shard import ShardRank, run_local
+def _run_sharded(G, spec, sh, counts, w, layers, regroup, fused=False):
+    from token_sparse_denoising_layer_b200.shard import ShardRank, link_local, run_local
 
     ranks = [ShardRank(r, G, sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]),
                        spec["T"], spec["budgets"], counts, shift=spec["shift"]) for r in range(G)]
+    if fused:
+        link_local(ranks)
     x0 = synth.latent(sh.N, 16, 9)
     g0 = synth.random_split(sh.N, counts, 9)
     for rk in ranks:
@@ -202,3 +204,117 @@ def test_sharded_conditioned_step(G):
     xr = O.run_loop(w, x0, g0, T, list(spec["budgets"]), counts,
                     O.sigma_schedule(T, spec["shift"]), sh.H, mods=mods, cross=cross)
     assert _rel(xs[0], xr) <= 2e-2
+
+
+# --------------------------------------------------------------------------- fused K|V exchange
+
+
+@pytest.mark.parametrize("N,D,a", [(700, 256, 333), (8192, 1536, 4097), (8192, 1536, 129)])
+@pytest.mark.parametrize("G", [1, 3, 8])
+def test_qkv_project_peers_writes_every_copy(N, D, a, G):
+    """hsa_qkv_project_peers: the same Q as hsa_qkv_project, bit for bit, and in
+    every one of the G cache pairs the same fresh rows at A and the copy's own
+    stale rows elsewhere; the rows also match the float64 oracle."""
+    need_gpu()
+    H = D // 128
+    ctx = abi.hsa_create(N=N, D=D, H=H, F=4 * D, L=1, T=1, budgets=[1], counts=[N])
+    w = synth.layer_weights(D, 64, 5)
+    x = synth.hidden_rows(N, D, 5)
+    idx = synth.random_active_set(N, a, 5)
+    u = torch.empty((a, D), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_ln_gather(ctx, dev(x), dev(idx), a, u)
+    wq = bf(w["w_qkv"])
+    ks, vs = synth.stale_kv(N, D, 5)
+    q1 = torch.empty((a, D), dtype=torch.bfloat16, device="cuda")
+    kc1, vc1 = bf(ks), bf(vs)
+    abi.hsa_qkv_project(ctx, wq, u, dev(idx), a, q1, kc1, vc1)
+    stale = [synth.stale_kv(N, D, 50 + g) for g in range(G)]
+    kcs = [bf(k) for k, _ in stale]
+    vcs = [bf(v) for _, v in stale]
+    q = torch.empty((a, D), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_qkv_project_peers(ctx, wq, u, dev(idx), a, q, kcs, vcs)
+    abi.hsa_sync_check(ctx)
+    assert torch.equal(q, q1)
+    rest = np.setdiff1d(np.arange(N), idx)
+    k1, v1 = host(kc1), host(vc1)
+    for g in range(G):
+        kg, vg = host(kcs[g]), host(vcs[g])
+        assert (kg[idx] == k1[idx]).all() and (vg[idx] == v1[idx]).all()
+        assert (kg[rest] == stale[g][0][rest]).all() and (vg[rest] == stale[g][1][rest]).all()
+    qkv = O.linear(O.layer_norm(x[idx]), w["w_qkv"])
+    assert normwise(host(q), qkv[:, :D]) <= BF16_TOL
+    assert normwise(k1[idx], qkv[:, D:2 * D]) <= BF16_TOL
+    assert normwise(v1[idx], qkv[:, 2 * D:]) <= BF16_TOL
+    ctx.close()
+
+
+def test_qkv_project_peers_rejects_bad_cache_lists():
+    need_gpu()
+    N, D = 256, 128
+    ctx = abi.hsa_create(N=N, D=D, H=1, F=512, L=1, T=1, budgets=[1], counts=[N])
+    u = torch.zeros((8, D), dtype=torch.bfloat16, device="cuda")
+    q = torch.empty_like(u)
+    wq = torch.zeros((3 * D, D), dtype=torch.bfloat16, device="cuda")
+    idx = torch.arange(8, dtype=torch.int32, device="cuda")
+    kc = torch.zeros((N, D), dtype=torch.bfloat16, device="cuda")
+    vc = torch.zeros_like(kc)
+    for ks, vs in (([], []), ([kc] * 9, [vc] * 9), ([kc, kc.data_ptr() + 2], [vc, vc]),
+                   ([kc, 0], [vc, vc])):
+        with pytest.raises(abi.HsaError) as e:
+            abi.hsa_qkv_project_peers(ctx, wq, u, idx, 8, q, ks, vs)
+        assert e.value.status == 1
+    abi.hsa_sync_check(ctx)
+    ctx.close()
+
+
+@pytest.mark.parametrize("G", [1, 2, 3])
+@pytest.mark.parametrize("regroup", [False, True])
+def test_sharded_fused_exchange_matches_all_gather(G, regroup):
+    """Ranks whose QKV epilogue writes every rank's cache end bit for bit where
+    the all-gather path ends, on every rank."""
+    need_gpu()
+    spec, sh, counts, w, layers = _model("tiny_dit")
+    _, _, xg, gg = _run_sharded(G, spec, sh, counts, w, layers, regroup)
+    _, _, xf, gf = _run_sharded(G, spec, sh, counts, w, layers, regroup, fused=True)
+    for r in range(G):
+        assert np.array_equal(xf[r], xg[0]) and np.array_equal(gf[r], gg[0])
+
+
+def test_sharded_fused_dit30_shapes_three_ranks():
+    need_gpu()
+    spec, sh, counts, w, layers = _model("dit30_1536", N=840, L=2)
+    _, _, xg, _ = _run_sharded(3, spec, sh, counts, w, layers, True)
+    _, _, xf, _ = _run_sharded(3, spec, sh, counts, w, layers, True, fused=True)
+    for r in range(3):
+        assert np.array_equal(xf[r], xg[0])
+
+
+def test_sharded_fused_world_of_one_through_symmetric_memory():
+    """The fused exchange across processes: caches in torch symmetric memory,
+    the barrier a one-element NCCL all-reduce.  A world of one equals the
+    in-process driver bit for bit."""
+    need_gpu()
+    import torch.distributed as dist
+
+    from token_sparse_denoising_layer_b200.shard import ShardRank, link_symmetric, run_dist
+
+    spec, sh, counts, w, layers = _model("tiny_dit")
+    x0, g0, xs, _ = _run_sharded(1, spec, sh, counts, w, layers, True)
+    store = dist.TCPStore("127.0.0.1", _free_port(), 1, True,
+                          timeout=datetime.timedelta(seconds=60))
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60),
+                            device_id=torch.device("cuda", torch.cuda.current_device()))
+    try:
+        rk = ShardRank(0, 1, sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]),
+                       spec["T"], spec["budgets"], counts, shift=spec["shift"])
+        link_symmetric(rk)
+        rk.reset(dev(x0), dev(g0))
+        for i in range(spec["T"]):
+            run_dist(rk.steps(i, True))
+        abi.hsa_sync_check(rk.ctx)
+        assert np.array_equal(host(rk.x), xs[0])
+        rk.close()
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()

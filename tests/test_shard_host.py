@@ -80,6 +80,34 @@ def _fake_steps(rank, G, N, D, plan, log):
         log.append(bool(torch.equal(v, want)))
 
 
+def _fake_fused_steps(rank, G, N, D, plan, caches, log):
+    """Stand-in for ShardRank.steps with the fused K|V exchange: the rank
+    writes its chunk's rows straight into every rank's copy of the layer's
+    cache (caches[layer, g] is rank g's copy), waits at the barrier, then
+    reads its own copy; one velocity reduction per iteration.  The next
+    layer writes other buffers, and the next iteration's writes come after
+    the reduction, which every rank reaches only after its reads."""
+    v = torch.zeros((N, 4))
+    sync = torch.zeros((1,), dtype=torch.int32)
+    for it, A in enumerate(plan):
+        a = len(A)
+        _, sl = shard_slices(a, G)
+        s0, nr = sl[rank]
+        for layer in range(2):
+            tag = 1000 * layer + 100000 * it
+            for g in range(G):
+                for p in range(s0, s0 + nr):
+                    caches[layer, g, A[p]] = float(p + tag)
+            yield ("barrier", sync)
+            got = caches[layer, rank, A, 0].numpy()
+            log.append(bool(np.array_equal(got, np.arange(a) + tag)))
+            log.append(bool((caches[layer, rank, A] == caches[layer, rank, A, :1]).all()))
+        v.zero_()
+        for p in range(s0, s0 + nr):
+            v[A[p]] = float(p + 1)
+        yield ("all_reduce_sum", v)
+
+
 def _plan(N, seed):
     r = np.random.default_rng(seed)
     sizes = [N, 1, 2, 3, N // 3, 5, N - 1]
@@ -92,6 +120,16 @@ def test_local_driver_exchanges(G):
     logs = [[] for _ in range(G)]
     plan = _plan(N, 3)
     run_local([_fake_steps(r, G, N, D, plan, logs[r]) for r in range(G)])
+    for lg in logs:
+        assert lg and all(lg)
+
+
+@pytest.mark.parametrize("G", [1, 2, 3])
+def test_local_driver_fused_exchange(G):
+    N, D = 37, 4
+    logs = [[] for _ in range(G)]
+    caches = torch.full((2, G, N, D), -7.0)
+    run_local([_fake_fused_steps(r, G, N, D, _plan(N, 3), caches, logs[r]) for r in range(G)])
     for lg in logs:
         assert lg and all(lg)
 
@@ -115,7 +153,7 @@ def _free_port():
     return port
 
 
-def _rank_main(rank, world, port, out):
+def _rank_main(rank, world, port, out, caches):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
                       WORLD_SIZE=str(world))
     sys.path.insert(0, ROOT)
@@ -128,6 +166,8 @@ def _rank_main(rank, world, port, out):
     dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
     log = []
     rd(_fake_steps(rank, world, 37, 4, _plan(37, 3), log))
+    # the fused exchange: every rank writes into all copies held in shared memory
+    rd(_fake_fused_steps(rank, world, 37, 4, _plan(37, 3), caches, log))
     dist.barrier()
     out.put((rank, len(log), all(log)))
     dist.destroy_process_group()
@@ -140,7 +180,9 @@ def test_gloo_ranks_exchange(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    caches = torch.full((2, world, 37, 4), -7.0).share_memory_()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q, caches))
+             for r in range(world)]
     for p in procs:
         p.start()
     for p in procs:

@@ -19,7 +19,7 @@ LIB_PATH = os.path.join(PKG, "libhsa.so")
 SYMBOLS = [
     "hsa_create", "hsa_destroy", "hsa_last_error", "hsa_set_stream", "hsa_sync_check",
     "hsa_selftest_timeout", "hsa_kernel_launches", "hsa_time_kernels", "hsa_kernel_times", "hsa_n_active", "hsa_schedule", "hsa_score", "hsa_select_from_score",
-    "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_linear", "hsa_kv_scatter", "hsa_kv_scatter_packed",
+    "hsa_select_groups", "hsa_ln_gather", "hsa_qkv_project", "hsa_qkv_project_peers", "hsa_linear", "hsa_kv_scatter", "hsa_kv_scatter_packed",
     "hsa_attention", "hsa_attention_kv", "hsa_out_proj_residual", "hsa_mlp_residual",
     "hsa_ln_gather_mod", "hsa_out_proj_residual_gated", "hsa_mlp_residual_mod",
     "hsa_layer_forward", "hsa_layer_forward_cond", "hsa_embed", "hsa_head", "hsa_euler_step", "hsa_euler_step_score", "hsa_step", "hsa_step_cond",
@@ -110,6 +110,7 @@ def load() -> ctypes.CDLL:
         "hsa_select_groups": (I, [P, P, P, P, P]),
         "hsa_ln_gather": (I, [P, P, P, I, P]),
         "hsa_qkv_project": (I, [P, P, P, P, I, P, P, P]),
+        "hsa_qkv_project_peers": (I, [P, P, P, P, I, P, ctypes.POINTER(P), ctypes.POINTER(P), I]),
         "hsa_linear": (I, [P, P, I, I, P, I, P]),
         "hsa_kv_scatter": (I, [P, P, P, P, I, P, P]),
         "hsa_kv_scatter_packed": (I, [P, P, P, I, P, P]),
@@ -149,6 +150,13 @@ def _p(t) -> Optional[int]:
     if not t.is_contiguous():
         raise ValueError("libhsa takes contiguous tensors")
     return t.data_ptr()
+
+
+def _addr(t) -> Optional[int]:
+    """Device address of a tensor, or an int taken as a device address as is."""
+    if isinstance(t, int):
+        return t
+    return _p(t)
 
 
 def _check(ctx, status: int) -> None:
@@ -260,6 +268,21 @@ def hsa_ln_gather(ctx: Context, x, idx, n: int, u) -> None:
 def hsa_qkv_project(ctx: Context, w_qkv, u, idx, n: int, q, k_cache, v_cache) -> None:
     _check(ctx.ptr, load().hsa_qkv_project(ctx.ptr, _p(w_qkv), _p(u), _p(idx), n, _p(q),
                                            _p(k_cache), _p(v_cache)))
+
+
+def hsa_qkv_project_peers(ctx: Context, w_qkv, u, idx, n: int, q, k_caches, v_caches) -> None:
+    """hsa_qkv_project writing the fresh K/V rows into every cache of the lists.
+
+    ``k_caches`` / ``v_caches`` are equal-length sequences of device buffers
+    (tensors) or raw device addresses (ints, e.g. peers' symmetric-memory
+    pointers)."""
+    if len(k_caches) != len(v_caches):
+        raise ValueError("k_caches and v_caches differ in length")
+    G = len(k_caches)
+    ks = (ctypes.c_void_p * max(G, 1))(*[_addr(t) for t in k_caches])
+    vs = (ctypes.c_void_p * max(G, 1))(*[_addr(t) for t in v_caches])
+    _check(ctx.ptr, load().hsa_qkv_project_peers(ctx.ptr, _p(w_qkv), _p(u), _p(idx), n, _p(q),
+                                                 ks, vs, G))
 
 
 def hsa_linear(ctx: Context, a, M: int, Kd: int, w, Ncols: int, out) -> None:

@@ -369,6 +369,46 @@ hsa_status hsa_qkv_project(hsa_ctx* ctx, const void* w_qkv, const void* u, const
   return launched(ctx, hsa::launch_gemm(ctx->c, g, &why), "qkv_project", why);
 }
 
+hsa_status hsa_qkv_project_peers(hsa_ctx* ctx, const void* w_qkv, const void* u,
+                                 const int32_t* idx, int n, void* q, void* const* k_caches,
+                                 void* const* v_caches, int n_caches) {
+  HSA_CHECK_CTX(ctx);
+  if (hsa_status st = check_n(ctx, n)) return st;
+  if (n_caches < 1 || n_caches > hsa::kMaxCaches)
+    return fail(ctx, HSA_ERR_INVALID_ARG, "n_caches outside [1, 8]");
+  if (k_caches == nullptr || v_caches == nullptr)
+    return fail(ctx, HSA_ERR_INVALID_ARG, "k_caches or v_caches is NULL");
+  for (int g = 0; g < n_caches; ++g) {
+    if (!aligned16(k_caches[g]) || !aligned16(v_caches[g]))
+      return fail(ctx, HSA_ERR_INVALID_ARG,
+                  "cache " + std::to_string(g) + " is NULL or not 16-byte aligned");
+  }
+  if (n == 0) return HSA_OK;
+  HSA_CHECK_PTR(ctx, w_qkv);
+  HSA_CHECK_PTR(ctx, u);
+  HSA_CHECK_PTR(ctx, idx);
+  HSA_CHECK_PTR(ctx, q);
+  const int D = ctx->c.cfg.D;
+  hsa::GemmArgs g{};
+  g.A = u;
+  g.B = w_qkv;
+  g.M = n;
+  g.Ncols = 3 * D;
+  g.Kd = D;
+  g.epi = hsa::EPI_QKV;
+  g.out = q;
+  g.ld_out = D;
+  g.n_caches = n_caches;
+  for (int c = 0; c < n_caches; ++c) {
+    g.k_caches[c] = k_caches[c];
+    g.v_caches[c] = v_caches[c];
+  }
+  g.idx = idx;
+  g.N = ctx->c.cfg.N;
+  std::string why;
+  return launched(ctx, hsa::launch_gemm(ctx->c, g, &why), "qkv_project_peers", why);
+}
+
 hsa_status hsa_kv_scatter(hsa_ctx* ctx, const void* k_rows, const void* v_rows,
                           const int32_t* idx, int n, void* k_cache, void* v_cache) {
   HSA_CHECK_CTX(ctx);

@@ -14,6 +14,7 @@
 namespace hsa {
 
 constexpr int kMaxGroups = 8;
+constexpr int kMaxCaches = 8;  // copies of a KV cache one QKV launch can write (ranks of a step)
 
 // Bits a kernel can set in the context's device flag (read by hsa_sync_check).
 enum : int { DEV_OK = 0, DEV_TIMEOUT = 1, DEV_BAD_INDEX = 2, DEV_BAD_SCORE = 4, DEV_BAD_GROUP = 8 };
@@ -157,6 +158,12 @@ struct GemmArgs {
   int ld_out;         // elements
   void* k_cache;      // EPI_QKV
   void* v_cache;      // EPI_QKV
+  // EPI_QKV into several copies of the caches (this GPU's and peers' over
+  // NVLink): when n_caches > 0, every fresh K/V row goes to rows idx[m] of
+  // k_caches[0 .. n_caches) and v_caches[..] instead of k_cache / v_cache
+  int n_caches = 0;
+  void* k_caches[kMaxCaches]{};
+  void* v_caches[kMaxCaches]{};
   float* x;           // EPI_RESID
   int ld_x;
   const float* gate = nullptr;  // EPI_RESID: x[.., j] += gate[j] * C (fp32 [Ncols]) if set

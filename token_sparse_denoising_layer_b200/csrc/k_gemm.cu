@@ -59,8 +59,9 @@ struct EpiParams {
   int M, Ncols, Kd, epi;
   __nv_bfloat16* out;
   int ld_out;
-  __nv_bfloat16* kc;
-  __nv_bfloat16* vc;
+  __nv_bfloat16* kc[kMaxCaches];  // EPI_QKV: n_caches copies of the K and V caches
+  __nv_bfloat16* vc[kMaxCaches];
+  int n_caches;
   float* x;
   int ld_x;
   const float* gate;
@@ -130,6 +131,16 @@ __device__ __forceinline__ F2 gelu_x2(F2 v) {
   const F2 he = mul_x2(t, F2{ex2_approx(s.x), ex2_approx(s.y)});  // erfc(z) / 2
   const F2 phi = F2{v.x >= 0.f ? 1.0f - he.x : he.x, v.y >= 0.f ? 1.0f - he.y : he.y};
   return mul_x2(v, phi);
+}
+
+// 32 fp32 accumulators -> 32 bf16 (rounded to nearest even) in four 16-byte words.
+__device__ __forceinline__ void pack_bf16x32(const uint32_t (&r)[32], uint4 (&w)[4]) {
+#pragma unroll
+  for (int v = 0; v < 4; ++v)
+    w[v] = make_uint4(pack_bf16(__uint_as_float(r[8 * v]), __uint_as_float(r[8 * v + 1])),
+                      pack_bf16(__uint_as_float(r[8 * v + 2]), __uint_as_float(r[8 * v + 3])),
+                      pack_bf16(__uint_as_float(r[8 * v + 4]), __uint_as_float(r[8 * v + 5])),
+                      pack_bf16(__uint_as_float(r[8 * v + 6]), __uint_as_float(r[8 * v + 7])));
 }
 
 // 32 fp32 accumulators -> 32 bf16 at dst (64 contiguous bytes, 16-byte aligned).
@@ -234,9 +245,24 @@ __device__ __forceinline__ void drain_tile(const EpiParams& p, uint32_t tbase, i
         const int cc = col - which * D;
         if (which == 0) {
           store_bf16x32<false>(p.out + static_cast<size_t>(m) * D + cc, cur);
-        } else if (dst_row >= 0) {
-          __nv_bfloat16* cache = which == 1 ? p.kc : p.vc;
+        } else if (dst_row >= 0 && p.n_caches == 1) {
+          __nv_bfloat16* cache = which == 1 ? p.kc[0] : p.vc[0];
           store_bf16x32<false>(cache + static_cast<size_t>(dst_row) * D + cc, cur);
+        } else if (dst_row >= 0) {
+          // the fresh row into every copy of this layer's cache (this GPU's,
+          // and peers' when a sharded step writes them directly)
+          uint4 w4[4];
+          pack_bf16x32(cur, w4);
+#pragma unroll
+          for (int g = 0; g < kMaxCaches; ++g) {
+            if (g >= p.n_caches) break;
+            __nv_bfloat16* cache = which == 1 ? p.kc[g] : p.vc[g];
+            uint4* d4 = reinterpret_cast<uint4*>(cache + static_cast<size_t>(dst_row) * D + cc);
+            d4[0] = w4[0];
+            d4[1] = w4[1];
+            d4[2] = w4[2];
+            d4[3] = w4[3];
+          }
         }
       }
     }
@@ -528,6 +554,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGemmThreads, 1)
   }
 }
 
+// The caches an EPI_QKV launch writes: the list when one is given, else the pair.
+void set_caches(EpiParams& p, const GemmArgs& a) {
+  if (a.n_caches > 0) {
+    p.n_caches = a.n_caches;
+    for (int g = 0; g < a.n_caches; ++g) {
+      p.kc[g] = static_cast<__nv_bfloat16*>(a.k_caches[g]);
+      p.vc[g] = static_cast<__nv_bfloat16*>(a.v_caches[g]);
+    }
+  } else {
+    p.n_caches = 1;
+    p.kc[0] = static_cast<__nv_bfloat16*>(a.k_cache);
+    p.vc[0] = static_cast<__nv_bfloat16*>(a.v_cache);
+  }
+}
+
 static_assert(kPairSmem <= 227 * 1024, "CTA-pair GEMM exceeds the shared memory of a CTA");
 static_assert(GemmCfg<256>::kSmem <= 227 * 1024 && GemmCfg<192>::kSmem <= 227 * 1024 &&
                   GemmCfg<128>::kSmem <= 227 * 1024,
@@ -544,8 +585,7 @@ cudaError_t launch_pair(const Ctx& c, const GemmArgs& a, std::string* why) {
   p.epi = a.epi;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.ld_out = a.ld_out;
-  p.kc = static_cast<__nv_bfloat16*>(a.k_cache);
-  p.vc = static_cast<__nv_bfloat16*>(a.v_cache);
+  set_caches(p, a);
   p.x = a.x;
   p.ld_x = a.ld_x;
   p.gate = a.gate;
@@ -577,8 +617,7 @@ cudaError_t launch_bn(const Ctx& c, const GemmArgs& a, std::string* why) {
   p.epi = a.epi;
   p.out = static_cast<__nv_bfloat16*>(a.out);
   p.ld_out = a.ld_out;
-  p.kc = static_cast<__nv_bfloat16*>(a.k_cache);
-  p.vc = static_cast<__nv_bfloat16*>(a.v_cache);
+  set_caches(p, a);
   p.x = a.x;
   p.ld_x = a.ld_x;
   p.gate = a.gate;

@@ -26,6 +26,19 @@ Per step on rank r:
   (replicated) -> re-grouping (replicated; deterministic, so the group ids
   stay identical on every rank).
 
+Fused K|V exchange (``link_local`` / ``link_symmetric``).  Instead of the
+Q and K|V GEMMs, the all-gather and the scatter, one QKV GEMM per layer
+(hsa_qkv_project_peers) stores every fresh K/V row of the rank's chunk
+straight into row A_i[m] of every rank's copy of the cache: its own through
+this GPU's memory, the others' through peer-mapped pointers over NVLink
+(stores only; nothing loads another GPU's memory).  A device-side barrier
+after it (a one-element all-reduce on the stream) keeps every rank's
+attention from reading its cache before all ranks' writes are complete.  The
+writes of step i + 1 cannot overtake a peer still reading step i's rows:
+they start after the velocity all-reduce of step i, which completes only
+once every rank has reached it, i.e. after all of that rank's step-i
+attention.
+
 Every step of the path runs in libhsa's kernels; the exchanges are
 collectives.  The step is written once, as a generator that yields each
 exchange; `run_dist` serves the requests with torch.distributed (NCCL on
@@ -62,7 +75,7 @@ def shard_slices(a: int, G: int) -> Tuple[int, List[Tuple[int, int]]]:
     return c, out
 
 
-Request = Tuple  # ("all_gather", send, recv) | ("all_reduce_sum", buf)
+Request = Tuple  # ("all_gather", send, recv) | ("all_reduce_sum", buf) | ("barrier", buf)
 
 
 class ShardRank:
@@ -107,12 +120,32 @@ class ShardRank:
         self.o = torch.empty((cmax, D), **bf)
         self.kv_send = torch.empty((cmax, 2 * D), **bf)
         self.kv_recv = torch.empty((G * cmax, 2 * D), **bf)
+        # fused exchange: layer l's cache of every rank, rank order (None: all-gather)
+        self.peer_k = None
+        self.peer_v = None
+        self.sync = torch.zeros((1,), dtype=torch.int32, device="cuda")
+        self._symm = None
         # W_qkv rows [0, D) project Q, rows [D, 3D) project K|V: contiguous views
         self.w_q = [lw[0][:D] for lw in layers]
         self.w_kv = [lw[0][D:] for lw in layers]
         self.layers = layers
         self.w_in, self.w_head = w_in, w_head
         self.sigmas = sigma_schedule(T, shift)
+
+    def link_peer_caches(self, k_caches, v_caches) -> None:
+        """Use the fused K|V exchange: ``k_caches[l]`` / ``v_caches[l]`` list
+        layer l's cache of every rank in rank order (tensors or device
+        addresses; this rank's entry is its own cache)."""
+        if len(k_caches) != self.L or len(v_caches) != self.L:
+            raise ValueError("need one list of caches per layer")
+        for l in range(self.L):
+            if len(k_caches[l]) != self.G or len(v_caches[l]) != self.G:
+                raise ValueError("need one cache per rank in every layer")
+            own = (abi._addr(k_caches[l][self.rank]), abi._addr(v_caches[l][self.rank]))
+            if own != (self.k_cache[l].data_ptr(), self.v_cache[l].data_ptr()):
+                raise ValueError("this rank's entry must be its own cache")
+        self.peer_k = [list(k) for k in k_caches]
+        self.peer_v = [list(v) for v in v_caches]
 
     def reset(self, x0, g0) -> None:
         """Start a run from latent x0 [N, 16] and group ids g0 [N] (same on every rank)."""
@@ -142,11 +175,16 @@ class ShardRank:
             m = None if mods is None else mods[l]   # rows shift_a, scale_a, gate_a, shift_m, ...
             row = (lambda r: None) if m is None else (lambda r, m=m: m[r])
             abi.hsa_ln_gather_mod(ctx, self.h, idx_r, nr, self.u, row(0), row(1))
-            abi.hsa_linear(ctx, self.u, nr, D, self.w_q[l], D, self.q)
-            abi.hsa_linear(ctx, self.u, nr, D, self.w_kv[l], 2 * D, self.kv_send)
-            yield ("all_gather", self.kv_send[:c], self.kv_recv[:self.G * c])
-            abi.hsa_kv_scatter_packed(ctx, self.kv_recv, self.active_idx, a, self.k_cache[l],
-                                      self.v_cache[l])
+            if self.peer_k is not None:
+                abi.hsa_qkv_project_peers(ctx, self.layers[l][0], self.u, idx_r, nr, self.q,
+                                          self.peer_k[l], self.peer_v[l])
+                yield ("barrier", self.sync)
+            else:
+                abi.hsa_linear(ctx, self.u, nr, D, self.w_q[l], D, self.q)
+                abi.hsa_linear(ctx, self.u, nr, D, self.w_kv[l], 2 * D, self.kv_send)
+                yield ("all_gather", self.kv_send[:c], self.kv_recv[:self.G * c])
+                abi.hsa_kv_scatter_packed(ctx, self.kv_recv, self.active_idx, a,
+                                          self.k_cache[l], self.v_cache[l])
             abi.hsa_attention(ctx, self.q, nr, self.k_cache[l], self.v_cache[l], self.o)
             abi.hsa_out_proj_residual_gated(ctx, w_o, self.o, idx_r, nr, self.h, row(2))
             xa = None if cross is None else cross[l]
@@ -175,6 +213,45 @@ class ShardRank:
 
     def close(self) -> None:
         self.ctx.close()
+        self.peer_k = self.peer_v = None
+        self._symm = None
+
+
+def link_local(ranks: Sequence[ShardRank]) -> None:
+    """Fused K|V exchange for ranks held in one process on one device: every
+    rank's QKV epilogue writes all ranks' caches directly."""
+    ks = [[rk.k_cache[l] for rk in ranks] for l in range(ranks[0].L)]
+    vs = [[rk.v_cache[l] for rk in ranks] for l in range(ranks[0].L)]
+    for rk in ranks:
+        rk.link_peer_caches(ks, vs)
+
+
+def link_symmetric(rk: ShardRank, group=None) -> None:
+    """Fused K|V exchange across processes: move this rank's caches into one
+    torch symmetric-memory buffer [L, 2, N, D] and take every rank's layer
+    caches from the peer mappings (collective over ``group``; NCCL ranks on
+    GPUs of one NVLink domain)."""
+    import torch
+    import torch.distributed as dist
+    import torch.distributed._symmetric_memory as symm
+
+    group = group or dist.group.WORLD
+    if dist.get_world_size(group) != rk.G or dist.get_rank(group) != rk.rank:
+        raise ValueError("group does not match the rank's (rank, G)")
+    L, N, D = rk.L, rk.N, rk.D
+    buf = symm.empty((L, 2, N, D), dtype=torch.bfloat16, device=torch.device("cuda"))
+    buf.zero_()
+    handle = symm.rendezvous(buf, group)
+    rk.k_cache = [buf[l, 0] for l in range(L)]
+    rk.v_cache = [buf[l, 1] for l in range(L)]
+    row = N * D * 2  # bytes of one cache
+    # the buffer sits at the same offset from every rank's mapped base
+    delta = buf.data_ptr() - int(handle.buffer_ptrs[rk.rank])
+    base = [int(p) + delta for p in handle.buffer_ptrs]
+    ks = [[b + (2 * l) * row for b in base] for l in range(L)]
+    vs = [[b + (2 * l + 1) * row for b in base] for l in range(L)]
+    rk._symm = (buf, handle)
+    rk.link_peer_caches(ks, vs)
 
 
 def _serve_dist(req: Request, group) -> None:
@@ -187,6 +264,9 @@ def _serve_dist(req: Request, group) -> None:
         else:
             dist.all_gather(list(recv.chunk(dist.get_world_size(group))), send, group=group)
     elif req[0] == "all_reduce_sum":
+        dist.all_reduce(req[1], op=dist.ReduceOp.SUM, group=group)
+    elif req[0] == "barrier":
+        # stream-ordered: completes only after every rank's earlier kernels
         dist.all_reduce(req[1], op=dist.ReduceOp.SUM, group=group)
     else:
         raise ValueError(f"unknown exchange {req[0]!r}")
@@ -220,6 +300,8 @@ def run_local(all_steps: Sequence[Iterator[Request]]) -> None:
             for _, _, recv in reqs:
                 for r, (_, send, _) in enumerate(reqs):
                     recv[r * send.shape[0]:(r + 1) * send.shape[0]].copy_(send)
+        elif op == "barrier":
+            pass  # one process, one stream: the writes are already ordered
         elif op == "all_reduce_sum":
             total = reqs[0][1].clone()
             for r in reqs[1:]:
