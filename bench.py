@@ -56,7 +56,8 @@ def parse():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--quick", action="store_true", help="skip the sub-benchmarks (profiling runs)")
     ap.add_argument("--profile-case", choices=["attention", "gemm", "euler", "rows", "tokens",
-                                                "embed_head", "gemm_epi", "gemm1"], default=None,
+                                                "embed_head", "gemm_epi", "gemm1", "qkv_peers"],
+                    default=None,
                     help="run three launches of one kernel at the workload shape and exit")
     return ap.parse_args()
 
@@ -1247,6 +1248,19 @@ def profile_case(name):
             abi.hsa_out_proj_residual(ctx, w_o, u, idx, N, x)
         for _ in range(2):
             abi.hsa_mlp_residual(ctx, w1, w2, x, idx, N)
+    elif name == "qkv_peers":
+        # one rank's QKV launch of a 4-way sequence-sharded step at 100% active
+        # (8190 rows of 32760), storing its fresh K/V rows into 4 cache copies
+        # (all in this GPU's memory here)
+        G, M = 4, N // 4
+        u = rnd(M, D).to(torch.bfloat16)
+        w_qkv = (rnd(3 * D, D) / D ** 0.5).to(torch.bfloat16)
+        kcs = [torch.zeros((N, D), dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+        vcs = [torch.zeros((N, D), dtype=torch.bfloat16, device="cuda") for _ in range(G)]
+        q = torch.empty((M, D), dtype=torch.bfloat16, device="cuda")
+        idx = torch.arange(M, dtype=torch.int32, device="cuda")  # rank 0's chunk of A_i
+        for _ in range(2):
+            abi.hsa_qkv_project_peers(ctx, w_qkv, u, idx, M, q, kcs, vcs)
     elif name == "gemm1":
         # the 1-CTA GEMM, as the tiny DiT (N = 256, D = 128, F = 512) runs it
         c1 = abi.hsa_create(N=256, D=128, H=2, F=512, L=1, T=1, budgets=[1], counts=[256])
