@@ -267,6 +267,41 @@ def test_qkv_project_peers_rejects_bad_cache_lists():
     ctx.close()
 
 
+def test_qkv_project_peers_skips_and_reports_bad_rows():
+    """Indices outside [0, N) are skipped in every copy and reported by
+    hsa_sync_check; the valid rows and Q are written as by hsa_qkv_project."""
+    need_gpu()
+    N, D, G = 256, 128, 3
+    ctx = abi.hsa_create(N=N, D=D, H=1, F=512, L=1, T=1, budgets=[1], counts=[N])
+    w = synth.layer_weights(D, 64, 7)
+    idx = np.array([1, 2, -1, 300, 5, 255], dtype=np.int32)
+    n = len(idx)
+    u = bf(synth.bf16_round(synth.rng(7).standard_normal((n, D), dtype=np.float32)))
+    wq = bf(w["w_qkv"])
+    ks, vs = synth.stale_kv(N, D, 7)
+    q1 = torch.empty((n, D), dtype=torch.bfloat16, device="cuda")
+    kc1, vc1 = bf(ks), bf(vs)
+    abi.hsa_qkv_project(ctx, wq, u, dev(idx), n, q1, kc1, vc1)
+    with pytest.raises(abi.HsaError) as e:
+        abi.hsa_sync_check(ctx)
+    assert e.value.status == 7
+    kcs = [bf(ks) for _ in range(G)]
+    vcs = [bf(vs) for _ in range(G)]
+    q = torch.empty((n, D), dtype=torch.bfloat16, device="cuda")
+    abi.hsa_qkv_project_peers(ctx, wq, u, dev(idx), n, q, kcs, vcs)
+    with pytest.raises(abi.HsaError) as e:
+        abi.hsa_sync_check(ctx)
+    assert e.value.status == 7
+    assert torch.equal(q, q1)
+    good = np.array([1, 2, 5, 255])
+    rest = np.setdiff1d(np.arange(N), good)
+    for g in range(G):
+        assert torch.equal(kcs[g], kc1) and torch.equal(vcs[g], vc1)
+        assert (host(kcs[g])[rest] == ks[rest]).all()
+    assert not (host(kc1)[good] == ks[good]).all()
+    ctx.close()
+
+
 @pytest.mark.parametrize("G", [1, 2, 3])
 @pytest.mark.parametrize("regroup", [False, True])
 def test_sharded_fused_exchange_matches_all_gather(G, regroup):

@@ -170,7 +170,8 @@ hsa_status hsa_create(const hsa_model_cfg* cfg, int T, const int* budgets, const
                    static_cast<size_t>(hsa::kMaxAttnParts) * 256 * 2 * sizeof(float));
   if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&x.cuts), 2 * hsa::kMaxGroups * sizeof(uint32_t));
   if (e == cudaSuccess) e = cudaMalloc(reinterpret_cast<void**>(&x.flag), sizeof(int));
-  if (e == cudaSuccess) e = cudaMemset(x.flag, 0, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemsetAsync(x.flag, 0, sizeof(int), x.stream);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(x.stream);
   if (e != cudaSuccess) {
     std::string msg = std::string("scratch allocation failed: ") + cudaGetErrorString(e);
     cudaGetLastError();
@@ -213,7 +214,9 @@ hsa_status hsa_sync_check(hsa_ctx* ctx) {
   e = cudaMemcpy(&flag, ctx->c.flag, sizeof(int), cudaMemcpyDeviceToHost);
   if (e != cudaSuccess) return cuda_fail(ctx, e, "read device flag");
   if (flag == 0) return HSA_OK;
-  cudaMemset(ctx->c.flag, 0, sizeof(int));
+  // cleared on the context's stream, so the next launch there sees it cleared
+  e = cudaMemsetAsync(ctx->c.flag, 0, sizeof(int), ctx->c.stream);
+  if (e != cudaSuccess) return cuda_fail(ctx, e, "clear device flag");
   std::string msg = "device check flag " + std::to_string(flag) + ":";
   if (flag & hsa::DEV_TIMEOUT) msg += " a bounded wait timed out;";
   if (flag & hsa::DEV_BAD_INDEX) msg += " an index was out of range;";
