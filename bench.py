@@ -1000,7 +1000,7 @@ def run_shard(args, rank, world, local, pg):
     import torch
 
     from token_sparse_denoising_layer_b200 import abi, synth
-    from token_sparse_denoising_layer_b200.shard import (ShardRank, link_local, link_symmetric,
+    from token_sparse_denoising_layer_b200.shard import (ShardRank, link_ipc, link_local,
                                                          run_dist, run_local)
 
     torch.cuda.set_device(local)
@@ -1015,7 +1015,7 @@ def run_shard(args, rank, world, local, pg):
                    spec["T"], spec["budgets"], counts, shift=spec["shift"])
     if args.kv_exchange == "peer":
         if pg is not None:
-            link_symmetric(rk, pg)
+            link_ipc(rk, pg)
         else:
             link_local([rk])
     x0 = torch.from_numpy(synth.latent(sh.N, 16, 0)).cuda()

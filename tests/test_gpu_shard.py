@@ -324,14 +324,14 @@ def test_sharded_fused_dit30_shapes_three_ranks():
         assert np.array_equal(xf[r], xg[0])
 
 
-def test_sharded_fused_world_of_one_through_symmetric_memory():
-    """The fused exchange across processes: caches in torch symmetric memory,
-    the barrier a one-element NCCL all-reduce.  A world of one equals the
+def test_sharded_fused_world_of_one_through_nccl():
+    """The fused exchange across processes (caches linked by CUDA IPC, the
+    barrier a one-element NCCL all-reduce) in a world of one equals the
     in-process driver bit for bit."""
     need_gpu()
     import torch.distributed as dist
 
-    from token_sparse_denoising_layer_b200.shard import ShardRank, link_symmetric, run_dist
+    from token_sparse_denoising_layer_b200.shard import ShardRank, link_ipc, run_dist
 
     spec, sh, counts, w, layers = _model("tiny_dit")
     x0, g0, xs, _ = _run_sharded(1, spec, sh, counts, w, layers, True)
@@ -343,7 +343,7 @@ def test_sharded_fused_world_of_one_through_symmetric_memory():
     try:
         rk = ShardRank(0, 1, sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]),
                        spec["T"], spec["budgets"], counts, shift=spec["shift"])
-        link_symmetric(rk)
+        link_ipc(rk)
         rk.reset(dev(x0), dev(g0))
         for i in range(spec["T"]):
             run_dist(rk.steps(i, True))
@@ -353,3 +353,86 @@ def test_sharded_fused_world_of_one_through_symmetric_memory():
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
+
+
+def _ipc_writer_rank(rank, port, out):
+    """One of two processes on GPU 0: both link their caches through CUDA IPC;
+    rank 1 runs the multi-copy QKV store into its own cache and rank 0's; rank
+    0 then checks its cache against a single-copy projection of its own."""
+    import sys
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    import datetime as dt
+
+    import torch as th
+    import torch.distributed as dist
+
+    from token_sparse_denoising_layer_b200 import abi as A
+    from token_sparse_denoising_layer_b200 import synth as S
+    from token_sparse_denoising_layer_b200.shard import open_peer_caches
+
+    ok, msg = False, ""
+    try:
+        th.cuda.set_device(0)
+        store = dist.TCPStore("127.0.0.1", port, 2, rank == 0, timeout=dt.timedelta(seconds=60))
+        dist.init_process_group("gloo", store=store, rank=rank, world_size=2,
+                                timeout=dt.timedelta(seconds=60))
+        N, D, a = 700, 256, 333
+        ctx = A.hsa_create(N=N, D=D, H=2, F=512, L=1, T=1, budgets=[1], counts=[N])
+        bf16 = lambda x: th.from_numpy(x).cuda().to(th.bfloat16)
+        ks0, vs0 = S.stale_kv(N, D, 60 + rank)
+        kc, vc = bf16(ks0), bf16(vs0)
+        kl, vl, keep = open_peer_caches([kc], [vc])
+        w = S.layer_weights(D, 64, 8)
+        idx = th.from_numpy(S.random_active_set(N, a, 8)).cuda()
+        u = bf16(S.bf16_round(S.rng(8).standard_normal((a, D), dtype=np.float32)))
+        wq = bf16(w["w_qkv"])
+        q = th.empty((a, D), dtype=th.bfloat16, device="cuda")
+        th.cuda.synchronize()
+        dist.barrier()
+        if rank == 1:
+            A.hsa_qkv_project_peers(ctx, wq, u, idx, a, q, kl[0], vl[0])
+            A.hsa_sync_check(ctx)
+            th.cuda.synchronize()
+        dist.barrier()  # rank 1's stores into rank 0's cache are complete
+        if rank == 0:
+            kr, vr = bf16(ks0), bf16(vs0)
+            A.hsa_qkv_project(ctx, wq, u, idx, a, q, kr, vr)
+            A.hsa_sync_check(ctx)
+            ok = bool(th.equal(kc, kr) and th.equal(vc, vr))
+            rest = np.setdiff1d(np.arange(N), idx.cpu().numpy())
+            ok = ok and bool((kc.float().cpu().numpy()[rest] == ks0[rest]).all())
+            msg = "rank 0 cache equals the single-copy projection" if ok else "mismatch"
+        else:
+            ok, msg = True, "writer"
+        dist.barrier()  # rank 0 has read its cache before the mappings go
+        del keep
+        th.cuda.synchronize()
+        dist.barrier()  # both mappings closed before either cache is freed
+        ctx.close()
+        dist.destroy_process_group()
+    except Exception as e:  # reported to the parent, which fails the test
+        msg = repr(e)
+    out.put((rank, ok, msg))
+
+
+def test_ipc_peer_stores_between_two_processes():
+    """The multi-copy QKV store through a CUDA IPC mapping of another process's
+    cache: two processes on one GPU, synchronised on the host only (no kernel
+    waits on the other process)."""
+    need_gpu()
+    import torch.multiprocessing as mp
+
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_ipc_writer_rank, args=(r, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=300) for _ in range(2))
+    for p in procs:
+        p.join(60)
+    print(res)
+    assert all(p.exitcode == 0 for p in procs)
+    assert [r for r, _, _ in res] == [0, 1]
+    assert all(ok for _, ok, _ in res), res

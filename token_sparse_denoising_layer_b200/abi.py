@@ -274,8 +274,8 @@ def hsa_qkv_project_peers(ctx: Context, w_qkv, u, idx, n: int, q, k_caches, v_ca
     """hsa_qkv_project writing the fresh K/V rows into every cache of the lists.
 
     ``k_caches`` / ``v_caches`` are equal-length sequences of device buffers
-    (tensors) or raw device addresses (ints, e.g. peers' symmetric-memory
-    pointers)."""
+    (tensors) or raw device addresses (ints, e.g. peers' caches mapped into this
+    process by CUDA IPC)."""
     if len(k_caches) != len(v_caches):
         raise ValueError("k_caches and v_caches differ in length")
     G = len(k_caches)

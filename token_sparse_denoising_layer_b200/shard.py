@@ -26,7 +26,7 @@ Per step on rank r:
   (replicated) -> re-grouping (replicated; deterministic, so the group ids
   stay identical on every rank).
 
-Fused K|V exchange (``link_local`` / ``link_symmetric``).  Instead of the
+Fused K|V exchange (``link_local`` / ``link_ipc``).  Instead of the
 Q and K|V GEMMs, the all-gather and the scatter, one QKV GEMM per layer
 (hsa_qkv_project_peers) stores every fresh K/V row of the rank's chunk
 straight into row A_i[m] of every rank's copy of the cache: its own through
@@ -37,7 +37,8 @@ attention from reading its cache before all ranks' writes are complete.  The
 writes of step i + 1 cannot overtake a peer still reading step i's rows:
 they start after the velocity all-reduce of step i, which completes only
 once every rank has reached it, i.e. after all of that rank's step-i
-attention.
+attention.  Across processes the peers' caches are reached through CUDA IPC
+mappings (point to point; no multicast object is created).
 
 Every step of the path runs in libhsa's kernels; the exchanges are
 collectives.  The step is written once, as a generator that yields each
@@ -124,7 +125,7 @@ class ShardRank:
         self.peer_k = None
         self.peer_v = None
         self.sync = torch.zeros((1,), dtype=torch.int32, device="cuda")
-        self._symm = None
+        self._peers = None
         # W_qkv rows [0, D) project Q, rows [D, 3D) project K|V: contiguous views
         self.w_q = [lw[0][:D] for lw in layers]
         self.w_kv = [lw[0][D:] for lw in layers]
@@ -214,7 +215,7 @@ class ShardRank:
     def close(self) -> None:
         self.ctx.close()
         self.peer_k = self.peer_v = None
-        self._symm = None
+        self._peers = None
 
 
 def link_local(ranks: Sequence[ShardRank]) -> None:
@@ -226,31 +227,49 @@ def link_local(ranks: Sequence[ShardRank]) -> None:
         rk.link_peer_caches(ks, vs)
 
 
-def link_symmetric(rk: ShardRank, group=None) -> None:
-    """Fused K|V exchange across processes: move this rank's caches into one
-    torch symmetric-memory buffer [L, 2, N, D] and take every rank's layer
-    caches from the peer mappings (collective over ``group``; NCCL ranks on
-    GPUs of one NVLink domain)."""
-    import torch
+def open_peer_caches(k_caches, v_caches, group=None):
+    """Every rank's copies of the per-layer caches as addresses valid in this
+    process (collective over ``group``): this rank's tensors as they are, the
+    other ranks' opened from their CUDA IPC handles, which map the peer's
+    memory point to point (no multicast object).  Returns (ks, vs, keep):
+    ks[l][r] and vs[l][r] for layer l of rank r, and the opened tensors, which
+    must outlive every launch that stores through their addresses."""
     import torch.distributed as dist
-    import torch.distributed._symmetric_memory as symm
+    from torch.multiprocessing.reductions import reduce_tensor
+
+    rank, G = dist.get_rank(group), dist.get_world_size(group)
+    L = len(k_caches)
+    mine = [(reduce_tensor(k), reduce_tensor(v)) for k, v in zip(k_caches, v_caches)]
+    everyone = [None] * G
+    dist.all_gather_object(everyone, mine, group=group)
+    ks = [[None] * G for _ in range(L)]
+    vs = [[None] * G for _ in range(L)]
+    keep = []
+    for r in range(G):
+        if len(everyone[r]) != L:
+            raise ValueError("ranks hold different numbers of layers")
+        for l in range(L):
+            if r == rank:
+                ks[l][r], vs[l][r] = k_caches[l], v_caches[l]
+                continue
+            (fk, ak), (fv, av) = everyone[r][l]
+            tk, tv = fk(*ak), fv(*av)
+            keep += [tk, tv]
+            ks[l][r], vs[l][r] = tk.data_ptr(), tv.data_ptr()
+    return ks, vs, keep
+
+
+def link_ipc(rk: ShardRank, group=None) -> None:
+    """Fused K|V exchange across processes: every rank's caches reached through
+    CUDA IPC peer mappings (collective over ``group``; ranks on GPUs of one
+    NVLink domain, one process each)."""
+    import torch.distributed as dist
 
     group = group or dist.group.WORLD
     if dist.get_world_size(group) != rk.G or dist.get_rank(group) != rk.rank:
         raise ValueError("group does not match the rank's (rank, G)")
-    L, N, D = rk.L, rk.N, rk.D
-    buf = symm.empty((L, 2, N, D), dtype=torch.bfloat16, device=torch.device("cuda"))
-    buf.zero_()
-    handle = symm.rendezvous(buf, group)
-    rk.k_cache = [buf[l, 0] for l in range(L)]
-    rk.v_cache = [buf[l, 1] for l in range(L)]
-    row = N * D * 2  # bytes of one cache
-    # the buffer sits at the same offset from every rank's mapped base
-    delta = buf.data_ptr() - int(handle.buffer_ptrs[rk.rank])
-    base = [int(p) + delta for p in handle.buffer_ptrs]
-    ks = [[b + (2 * l) * row for b in base] for l in range(L)]
-    vs = [[b + (2 * l + 1) * row for b in base] for l in range(L)]
-    rk._symm = (buf, handle)
+    ks, vs, keep = open_peer_caches(rk.k_cache, rk.v_cache, group)
+    rk._peers = keep
     rk.link_peer_caches(ks, vs)
 
 
