@@ -155,6 +155,50 @@ def test_layer_forward_empty_active_set_is_noop():
     assert (host(xd) == x).all()
 
 
+def test_every_row_entry_point_with_no_rows_launches_nothing():
+    """n = 0 active rows (M = 0 for the plain GEMM) is a valid no-op for every
+    per-row entry point: status OK, no kernel launched, no buffer touched."""
+    need_gpu()
+    N, D, H, F = 256, 128, 2, 512
+    ctx = _ctx(N, D, H, F)
+    w = synth.layer_weights(D, F, 9)
+    wq, wo, w1, w2 = (bf(w[k]) for k in ("w_qkv", "w_o", "w_1", "w_2"))
+    x = dev(synth.hidden_rows(N, D, 9))
+    x0 = x.clone()
+    kc, vc = (bf(c) for c in synth.stale_kv(N, D, 9))
+    k0, v0 = kc.clone(), vc.clone()
+    idx = dev(np.arange(4, dtype=np.int32))
+    rows = torch.full((4, D), 7.0, dtype=torch.bfloat16, device="cuda")
+    rows0 = rows.clone()
+    mod = torch.zeros((D,), dtype=torch.float32, device="cuda")
+    w_in = torch.ones((D, 16), dtype=torch.float32, device="cuda")
+    w_head = torch.ones((16, D), dtype=torch.float32, device="cuda")
+    lat = torch.ones((N, 16), dtype=torch.float32, device="cuda")
+    vf = torch.full((N, 16), 3.0, dtype=torch.float32, device="cuda")
+    vf0 = vf.clone()
+    before = abi.hsa_kernel_launches(ctx)
+    abi.hsa_ln_gather(ctx, x, idx, 0, rows)
+    abi.hsa_ln_gather_mod(ctx, x, idx, 0, rows, mod, mod)
+    abi.hsa_qkv_project(ctx, wq, rows, idx, 0, rows, kc, vc)
+    abi.hsa_qkv_project_peers(ctx, wq, rows, idx, 0, rows, [kc, kc.clone()], [vc, vc.clone()])
+    abi.hsa_linear(ctx, rows, 0, D, wq, 3 * D, rows)
+    abi.hsa_kv_scatter(ctx, rows, rows, idx, 0, kc, vc)
+    abi.hsa_kv_scatter_packed(ctx, rows, idx, 0, kc, vc)
+    abi.hsa_attention(ctx, rows, 0, kc, vc, rows)
+    abi.hsa_attention_kv(ctx, rows, 0, kc, vc, 16, rows)
+    abi.hsa_out_proj_residual(ctx, wo, rows, idx, 0, x)
+    abi.hsa_out_proj_residual_gated(ctx, wo, rows, idx, 0, x, mod)
+    abi.hsa_mlp_residual(ctx, w1, w2, x, idx, 0)
+    abi.hsa_mlp_residual_mod(ctx, w1, w2, x, idx, 0, mod, mod, mod)
+    abi.hsa_embed(ctx, w_in, lat, idx, 0, x)
+    abi.hsa_head(ctx, w_head, x, idx, 0, vf)
+    abi.hsa_sync_check(ctx)
+    assert abi.hsa_kernel_launches(ctx) == before
+    assert torch.equal(x, x0) and torch.equal(kc, k0) and torch.equal(vc, v0)
+    assert torch.equal(rows, rows0) and torch.equal(vf, vf0)
+    ctx.close()
+
+
 def test_bad_index_is_reported_not_faulted():
     need_gpu()
     N, D = 256, 128
