@@ -222,7 +222,7 @@ hsa_status hsa_qkv_project(hsa_ctx* ctx, const void* w_qkv, const void* u, const
  *   w_qkv, u, idx, q as hsa_qkv_project;
  *   k_caches, v_caches (HOST arrays of n_caches pointers, borrowed for the
  *   call): device bf16 [N, D] caches, each on this GPU or a peer GPU's memory
- *   mapped into this process (P2P or symmetric memory); 1 <= n_caches <= 8.
+ *   mapped into this process (CUDA IPC or peer access); 1 <= n_caches <= 8.
  * The launch only stores to peer memory (no load reads another GPU).  The
  * caller orders it against the peers' readers: no peer may read the rows
  * before this launch completes (a device-side barrier on the stream after
