@@ -155,15 +155,15 @@ def test_sharded_world_of_one_through_nccl():
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("G", [1, 2, 3])
-def test_sharded_conditioned_step(G):
+@pytest.mark.parametrize("G,fused", [(1, False), (2, False), (3, False), (2, True), (3, True)])
+def test_sharded_conditioned_step(G, fused):
     """Conditioned blocks (per-iteration modulation of every layer, text
     cross-attention in every layer) in the sharded step: every rank ends with
     the same latent bit for bit, equal to the single-GPU conditioned loop
     (hsa_step_cond) within rounding, and to the float64 oracle within 2e-2."""
     need_gpu()
     from token_sparse_denoising_layer_b200.loop import HsaLoop
-    from token_sparse_denoising_layer_b200.shard import ShardRank, run_local
+    from token_sparse_denoising_layer_b200.shard import ShardRank, link_local, run_local
 
     spec, sh, counts, w, layers = _model("tiny_dit")
     T, L = spec["T"], sh.L
@@ -178,6 +178,8 @@ def test_sharded_conditioned_step(G):
     g0 = synth.random_split(sh.N, counts, 9)
     ranks = [ShardRank(r, G, sh.N, sh.D, sh.H, sh.F, layers, dev(w["w_in"]), dev(w["w_head"]),
                        T, spec["budgets"], counts, shift=spec["shift"]) for r in range(G)]
+    if fused:
+        link_local(ranks)
     for rk in ranks:
         rk.reset(dev(x0), dev(g0))
     for i in range(T):
