@@ -361,6 +361,7 @@ def _ipc_writer_rank(rank, port, out):
     """One of two processes on GPU 0: both link their caches through CUDA IPC;
     rank 1 runs the multi-copy QKV store into its own cache and rank 0's; rank
     0 then checks its cache against a single-copy projection of its own."""
+    import gc
     import sys
 
     sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
@@ -408,9 +409,12 @@ def _ipc_writer_rank(rank, port, out):
         else:
             ok, msg = True, "writer"
         dist.barrier()  # rank 0 has read its cache before the mappings go
-        del keep
+        del keep, kl, vl
+        gc.collect()
         th.cuda.synchronize()
-        dist.barrier()  # both mappings closed before either cache is freed
+        dist.barrier()  # both mappings released before either cache is freed
+        th.cuda.ipc_collect()
+        dist.barrier()
         ctx.close()
         dist.destroy_process_group()
     except Exception as e:  # reported to the parent, which fails the test
